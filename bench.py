@@ -1,0 +1,425 @@
+"""Throughput of the ButterflyMoE expert forward (router + forward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One JSON line on rank 0.  A step is one router + forward pass over one batch
+of the named synthetic workload (default: d=512, N=256 experts, top-2,
+T=16384 bf16 tokens).  Inputs are resident in HBM before the timed region;
+L2 is flushed (a 512 MiB write) between timed steps, outside the timed
+intervals.  Each step is timed with CUDA events on the launching stream; the
+total is the max over ranks.  With N > 1 GPUs every rank runs its own batch
+(tokens shard with no collective on the data path; weights are replicated):
+"scaling": "weak".
+
+``--impl reference`` times the CPU float64 oracle (test infrastructure) on the
+host cores instead, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "routed tokens/sec (bf16, d=512, N=256, top-2)"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def physical_gpu_index(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v for v in vis.split(",") if v.strip()]
+    if ids and local < len(ids) and ids[local].strip().isdigit():
+        return int(ids[local])
+    return local
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu_index)], stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, mx, pw = [], [], []
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                    pw.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        # "under load": samples within the busiest part of the run
+        top = sorted(sm)
+        load = [s for s in sm if s >= 0.5 * top[-1]] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx), "power_w_max": max(pw),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic cost of each kernel, per launch (the roofline numerators)
+# ---------------------------------------------------------------------------
+def kernel_costs(wl, tables_bytes):
+    d, N, k, T = wl.d, wl.n_experts, wl.k, wl.tokens
+    R = T * k
+    L = wl.stages
+    xb = 2 if wl.dtype == "bf16" else 4
+    return {
+        # GEMM: 2 R d^2 flops on the tensor cores
+        "ternary_gemm_tc": ("tensor", 2.0 * R * d * d, "TFLOP/s"),
+        "ternary_gemm_simt": ("alu", 2.0 * R * d * d, "TFLOP/s"),
+        # router product on the CUDA cores: 2 T N d flops
+        "router_logits_simt": ("alu", 2.0 * T * N * d, "TFLOP/s"),
+        # pre-rotation: x rows gathered (R rows) + X_rot written + the theta table
+        "pre_rotate": ("hbm", R * d * xb + R * d * xb + tables_bytes, "GB/s"),
+        # post-rotation: Z read (fp32) + slots written (fp32) + the phi table
+        "post_rotate": ("hbm", R * d * 4 + R * d * 4 + tables_bytes, "GB/s"),
+        "combine": ("hbm", R * d * 4 + T * d * xb, "GB/s"),
+        "rot_table": ("hbm", N * L * (d // 2) * 4 + tables_bytes, "GB/s"),
+        "router_topk": ("hbm", T * N * 4 + T * k * 8, "GB/s"),
+    }
+
+
+def alu_peak_tflops(sm_mhz):
+    return SM_COUNT * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+
+
+# ---------------------------------------------------------------------------
+# The CPU oracle as the baseline (host cores)
+# ---------------------------------------------------------------------------
+def oracle_expert_slice(inp, experts):
+    """Oracle output for every routed row whose expert is in ``experts``
+    (routing over all tokens, dense experts, per-expert products).
+    Returns (rows evaluated, seconds)."""
+    from oracle import bfmoe_oracle as O
+    t0 = time.perf_counter()
+    x = inp.x_f64()
+    idx, gates, _, _ = O.route(x, inp.w_gate, inp.bias, inp.wl.k)
+    flat = idx.reshape(-1)
+    k = inp.wl.k
+    y = np.zeros_like(x)
+    rows = 0
+    for e in experts:
+        r = np.nonzero(flat == e)[0]
+        if r.size == 0:
+            continue
+        We = O.expert_matrix(inp.w_base, inp.alpha, inp.theta[e], inp.phi[e])
+        t, j = r // k, r % k
+        np.add.at(y, t, gates[t, j][:, None] * (x[t] @ We.T))
+        rows += r.size
+    return rows, time.perf_counter() - t0
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        th = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        th = os.cpu_count() or 1
+    return th
+
+
+def cpu_baseline(inp, frac_experts: float):
+    N = inp.wl.n_experts
+    n = max(1, int(round(N * frac_experts)))
+    rows, sec = oracle_expert_slice(inp, range(n))
+    return {"value": (rows / inp.wl.k) / sec, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{inp.wl.describe()}: all tokens routed, rows of experts 0..{n - 1} "
+                      f"({rows} rows = {rows / inp.wl.k:.0f} token-equivalents) formed densely and multiplied; "
+                      f"{sec:.1f} s"}
+
+
+def run_reference(args, wl):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = W.generate(wl, seed=0)
+    N = wl.n_experts
+    per = max(1, N // 16)
+    times, units = [], []
+    for step in range(args.warmup + args.steps):
+        lo = (step * per) % N
+        rows, sec = oracle_expert_slice(inp, range(lo, min(N, lo + per)))
+        if step >= args.warmup:
+            times.append(sec)
+            units.append(rows / wl.k)
+    total = sum(times)
+    value = sum(units) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(wl, "n/a (host)"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"each step: all {wl.tokens} tokens routed, rows of {per} consecutive "
+                                   f"experts (of {N}) formed densely and multiplied"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, l2):
+    return {"workload": wl.name, "d": wl.d, "n_experts": wl.n_experts, "k": wl.k, "tokens": wl.tokens,
+            "x_dtype": wl.dtype, "routed_rows": wl.tokens * wl.k, "l2": l2, "parallelism": "token shards"}
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from ternary_butterfly_experts_b200 import build as b
+    if rank == 0:
+        b.build()
+    if world > 1:
+        dist.barrier()
+    import ternary_butterfly_experts_b200 as B
+
+    peaks, peak_src = load_peaks()
+    inp = W.generate(wl, seed=0)
+    layer = B.Layer.from_host(inp.w_base, inp.alpha, inp.theta, inp.phi, device=dev)
+    wg = torch.from_numpy(inp.w_gate).to(dev)
+    bias = None if inp.bias is None else torch.from_numpy(inp.bias).to(dev)
+    x = inp.x.to(dev).contiguous()
+    model = B.ButterflyMoE(layer, wg, bias, wl.k, wl.tokens, x.dtype)
+    y = torch.empty_like(x)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        model(x, y=y)
+
+    def timed(n, fn, flush_l2=True):
+        evs = []
+        for _ in range(n):
+            if flush_l2:
+                flush.fill_(1.0)
+            a = torch.cuda.Event(enable_timing=True)
+            bb = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            bb.record(stream)
+            evs.append((a, bb))
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(bb) for a, bb in evs)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    B.bfmoe_check_device_error()
+
+    # --- timed region ---------------------------------------------------------
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = B.bfmoe_launch_count()
+    with ClockSampler(physical_gpu_index(local)) as clocks:
+        total_ms = timed(args.steps, step)
+    launches = B.bfmoe_launch_count() - launches0
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    B.bfmoe_check_device_error()
+
+    # --- per-kernel device times (same steps again, each launch bracketed) ------
+    B.bfmoe_profile_enable(True)
+    prof_ms = timed(args.steps, step)
+    kt = B.bfmoe_profile_collect()
+    B.bfmoe_profile_enable(False)
+
+    # --- end to end through host buffers ----------------------------------------
+    x_host = inp.x.pin_memory()
+    y_host = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    for _ in range(2):
+        model.forward_host(x_host, y_host)
+    e2e_ms = timed(args.steps, lambda: model.forward_host(x_host, y_host))
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    if rank == 0:
+        clk = clocks.summary()
+        T = wl.tokens
+        value = T * world * args.steps / (total_ms / 1e3)
+        L = wl.stages
+        tables = 2 * wl.n_experts * L * (wl.d // 2) * 8
+        costs = kernel_costs(wl, tables // 2)
+        kernels = {}
+        for name, (n, ms) in kt.items():
+            entry = {"launches": n, "total_ms": ms, "share": ms / max(1e-9, sum(v[1] for v in kt.values())),
+                     "avg_us": 1e3 * ms / n}
+            kernels[name] = entry
+        dom = max(kt.items(), key=lambda kv: kv[1][1])[0]
+        roof = roofline_entry(dom, kt[dom], costs, peaks, clk)
+        flops = 2.0 * T * wl.k * wl.d ** 2
+        bytes_alg = algorithmic_bytes(wl)
+        t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_alg / (peaks["hbm_gbs"] * 1e9))
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": workload_config(wl, "flushed between steps (512 MiB write, outside the timed intervals)"),
+            "roofline": roof,
+            "path_roofline": {"time_us": t_roof * 1e6, "achieved_us": 1e3 * total_ms / args.steps,
+                              "frac": t_roof / (total_ms / args.steps / 1e3),
+                              "formula": "max(2 T k d^2 / bf16 peak, algorithmic bytes / HBM BW)",
+                              "peak_source": peak_src},
+            "kernels": kernels,
+            "profiled_pass_ms_per_step": prof_ms / args.steps,
+            "cpu_baseline": None,
+            "e2e": {"value": T * world * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                    "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(inp, args.cpu_fraction)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def algorithmic_bytes(wl):
+    """x read once, y written once, packed base, angles, router weights and
+    bias, routing outputs."""
+    d, N, k, T = wl.d, wl.n_experts, wl.k, wl.tokens
+    xb = 2 if wl.dtype == "bf16" else 4
+    return (2 * T * d * xb + d * d // 4 + 2 * N * wl.stages * (d // 2) * 4 + N * d * 4 + N * 4
+            + T * k * 8)
+
+
+def roofline_entry(name, kt_entry, costs, peaks, clk):
+    n, ms = kt_entry
+    avg_s = ms / n / 1e3
+    bound, work, unit = costs.get(name, ("hbm", float("nan"), "GB/s"))
+    if bound == "tensor":
+        achieved = work / avg_s / 1e12
+        peak = peaks["bf16_tflops"]
+        src = "bf16_tflops (measured burst)"
+    elif bound == "alu":
+        achieved = work / avg_s / 1e12
+        mhz = peaks.get("sm_max_mhz", 1965.0)
+        peak = alu_peak_tflops(mhz)
+        src = f"fp32 FMA: {SM_COUNT} SMs x {FP32_LANES_PER_SM} lanes x 2 x {mhz:.0f} MHz"
+    else:
+        achieved = work / avg_s / 1e9
+        peak = peaks["hbm_gbs"]
+        src = "hbm_gbs (measured copy)"
+    return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": None, "avg_launch_us": avg_s * 1e6,
+            "work_per_launch": work, "peak_source": src}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-fraction", type=float, default=1.0,
+                    help="fraction of the experts whose rows the CPU baseline evaluates")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    wl = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

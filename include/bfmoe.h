@@ -1,0 +1,187 @@
+/*
+ * bfmoe.h - C ABI of the ButterflyMoE expert forward on NVIDIA B200 (sm_100a).
+ *
+ * The method (ButterflyMoE: sub-linear ternary experts via structured
+ * butterfly orbits; gist.science technical summary, sections 2.1-2.3):
+ * every expert is W_i = B(phi_i) . W_base . B(theta_i)^T, where W_base is one
+ * d x d ternary {-1, 0, +1} matrix shared by all N experts (scaled here by one
+ * float alpha) and B(.) is a butterfly of log2(d) stages of d/2 Givens
+ * rotations, one angle per rotation.  Inference never forms W_i: a token x
+ * routed to experts e_0..e_{k-1} with gates g_j gets
+ *     y = sum_j g_j * B(phi_{e_j}) (alpha * W_base (B(theta_{e_j})^T x)).
+ *
+ * Conventions shared by every call (the pages leave them open):
+ *  - stage s (stride h = 2^s) rotates the pairs (i, i+h) with bit s of i
+ *    clear; its rotations are numbered by ascending i; the 2x2 block is
+ *    [[cos a, -sin a], [sin a, cos a]]; B = S_{L-1} ... S_1 S_0, so stage 0
+ *    acts first; B^T is the literal transpose (stages L-1 ... 0, blocks
+ *    transposed).
+ *  - W_base[o][i]: row o is the output, column i the input (y = W x).
+ *  - angles are float32 [N][log2 d][d/2]; tokens and outputs are row-major
+ *    [T][d] in float32 or bfloat16.
+ *  - routed row r = t*k + j is slot j of token t.
+ *
+ * Memory: every pointer is caller-owned.  Pointers named "device" must be
+ * device memory of the current device; the library allocates nothing per
+ * call.  A call only enqueues work on `stream` (no host synchronisation)
+ * unless its comment says it synchronises.
+ *
+ * Errors: every int-returning call returns a bfmoe_status.  Argument checks
+ * run on the host before any launch; on failure nothing is launched and
+ * bfmoe_last_error() (thread-local) describes the problem.  Device-side checks
+ * (an index out of range in caller-provided routing arrays, a bounded wait
+ * that ran out) never trap: the kernel skips the bad access, records a code
+ * in a device error word and returns; bfmoe_check_device_error() reads it.
+ */
+#ifndef BFMOE_H
+#define BFMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The same handle as cudaStream_t (NULL = the legacy default stream). */
+typedef struct CUstream_st* bfmoe_stream_t;
+
+typedef enum {
+  BFMOE_OK = 0,
+  BFMOE_EINVAL = 1,           /* null pointer, size or shape out of range      */
+  BFMOE_ENOT_TERNARY = 2,     /* a base weight outside {-1, 0, +1}             */
+  BFMOE_EUNSUPPORTED = 3,     /* well-formed but outside the supported range   */
+  BFMOE_EWORKSPACE = 4,       /* workspace missing, too small or misaligned    */
+  BFMOE_ECUDA = 5,            /* a CUDA runtime call failed                    */
+  BFMOE_EDEVICE_TIMEOUT = 6,  /* a device-side bounded wait ran out            */
+  BFMOE_EDEVICE_BOUNDS = 7    /* a device-side index check failed              */
+} bfmoe_status;
+
+typedef enum { BFMOE_F32 = 0, BFMOE_BF16 = 1 } bfmoe_dtype;
+
+/* Supported ranges. */
+#define BFMOE_MAX_D 4096        /* d: power of two, 4 <= d <= 4096         */
+#define BFMOE_MAX_EXPERTS 4096  /* N: 1 <= N <= 4096                       */
+#define BFMOE_MAX_K 8           /* k: 1 <= k <= min(8, N)                  */
+
+/* One ButterflyMoE layer (all pointers device, caller-owned, read-only). */
+typedef struct {
+  int d;                      /* width; power of two in [4, BFMOE_MAX_D]           */
+  int n_experts;              /* N                                                  */
+  const uint32_t* w_packed;   /* [d][max(1, d/16)] 2-bit codes (bfmoe_pack_base)   */
+  float alpha;                /* scale of the ternary base                          */
+  const float* theta;         /* [N][log2 d][d/2] input-side angles  (B(theta)^T)  */
+  const float* phi;           /* [N][log2 d][d/2] output-side angles (B(phi))      */
+} bfmoe_layer;
+
+/*
+ * Pack the shared ternary base (one-time weight load).
+ * The pages store W_base at 1.58 bits per weight (technical summary, 2.1);
+ * this storage spends 2 bits: 0 -> 00, +1 -> 01, -1 -> 11 (10 is never
+ * written and reads as 0), 16 codes per uint32, row-major, column i of a word
+ * at bits 2*(i mod 16).  Row length is max(1, d/16) words.
+ *   w        device int8 [d][d], values in {-1, 0, +1}
+ *   w_packed device uint32 [d][max(1, d/16)] (written)
+ * Synchronises `stream` to report BFMOE_ENOT_TERNARY (then w_packed holds 0
+ * for every invalid weight).
+ */
+int bfmoe_pack_base(const int8_t* w, int d, uint32_t* w_packed, bfmoe_stream_t stream);
+
+/*
+ * Expand the packed base to the exact bfloat16 matrix the tensor-core GEMM
+ * multiplies by (checking aid for the 2-bit code).
+ *   w_bf16   device uint16 [d][d] (bfloat16 bit patterns 0x0000, 0x3F80, 0xBF80)
+ */
+int bfmoe_unpack_base(const uint32_t* w_packed, int d, uint16_t* w_bf16, bfmoe_stream_t stream);
+
+/*
+ * Router: logits l = x W_g^T (+ b) in float32; top-k experts per token by
+ * descending logit, the lower expert index first on equal logits (and NaN
+ * below every number); gates g_j = exp(l_{e_j} - l_{e_0}) / sum_j' exp(...)
+ * (softmax over all N, top-k, renormalised); then the token-to-expert
+ * buckets.  The pages only define mixture-of-experts selection in general
+ * (signalfieldnotes ButterflyMoE article, glossary "Mixtures of Experts").
+ *   x         device [T][d], dtype x_dtype
+ *   w_gate    device float [N][d];  bias: device float [N] or NULL
+ *   idx       device int32 [T][k] (written): experts, slot order
+ *   gates     device float [T][k] (written)
+ *   counts    device int32 [N]    (written): rows per expert
+ *   offsets   device int32 [N+1]  (written): exclusive prefix sum of counts
+ *   rows      device int32 [T*k]  (written): expert by expert, that expert's
+ *             routed rows r = t*k + j in ascending token order
+ *   ws        device scratch of at least bfmoe_workspace_size(...) bytes,
+ *             256-byte aligned
+ * T = 0 is allowed (counts and offsets are zeroed).
+ */
+int bfmoe_router_topk(const void* x, int x_dtype, int T, int d,
+                      const float* w_gate, const float* bias, int n_experts, int k,
+                      int32_t* idx, float* gates,
+                      int32_t* counts, int32_t* offsets, int32_t* rows,
+                      void* ws, size_t ws_bytes, bfmoe_stream_t stream);
+
+/*
+ * Expert forward without forming any expert (technical summary, 2.3):
+ * for every routed row, B(theta_e)^T x_t, then alpha * W_base (.), then
+ * B(phi_e) (.), times the gate; the k rows of a token are summed in slot
+ * order in float32 and rounded once to the output dtype.
+ *   layer     weights (see bfmoe_layer)
+ *   x         device [T][d], dtype x_dtype
+ *   idx, gates, offsets, rows: as written by bfmoe_router_topk (any routing
+ *             with k distinct experts per token and consistent buckets)
+ *   y         device [T][d], dtype x_dtype (written)
+ *   ws        device scratch, bfmoe_workspace_size(d, N, T, k, x_dtype) bytes
+ * The bfloat16 path rounds B(theta)^T x to bfloat16 before the tensor-core
+ * product (the ternary weights are exact in bfloat16); rotations, the
+ * product's accumulation, the gates and the combine are float32.  The float32
+ * path keeps every intermediate in float32.
+ */
+int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, int k,
+                  const int32_t* idx, const float* gates,
+                  const int32_t* offsets, const int32_t* rows,
+                  void* y, void* ws, size_t ws_bytes, bfmoe_stream_t stream);
+
+/*
+ * Form expert e densely, alpha * B(phi_e) . W_base . B(theta_e)^T, in float32
+ * (technical summary, 2.1).  For checking only.
+ *   w_out     device float [d][d] (written), row = output
+ */
+int bfmoe_materialize_expert(const bfmoe_layer* layer, int e, float* w_out,
+                             bfmoe_stream_t stream);
+
+/* Scratch bytes that bfmoe_router_topk and bfmoe_forward need for these
+ * sizes (one buffer serves both; calls on one stream may share it).
+ * Returns 0 for invalid sizes. */
+size_t bfmoe_workspace_size(int d, int n_experts, int T, int k, int x_dtype);
+
+/* Thread-local description of the last failed call ("" if none). */
+const char* bfmoe_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns BFMOE_OK, BFMOE_EDEVICE_TIMEOUT,
+ * BFMOE_EDEVICE_BOUNDS or BFMOE_ECUDA. */
+int bfmoe_check_device_error(bfmoe_stream_t stream);
+
+/* ---- tracing ------------------------------------------------------------ */
+
+/* Number of kernels this library has launched in this process. */
+unsigned long long bfmoe_launch_count(void);
+
+typedef struct {
+  char name[48];        /* kernel name                              */
+  int launches;         /* launches recorded since profiling began  */
+  double total_ms;      /* summed device time (CUDA events)          */
+} bfmoe_kernel_time;
+
+/* While enabled, every launch is bracketed by two CUDA events recorded on
+ * its own stream.  Enabling discards earlier records. */
+int bfmoe_profile_enable(int on);
+
+/* Synchronises the recorded events and writes per-kernel totals
+ * (at most `max` entries; *n_out = entries written).  Clears the records. */
+int bfmoe_profile_collect(bfmoe_kernel_time* out, int max, int* n_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BFMOE_H */

@@ -1,0 +1,563 @@
+// Host side of the ButterflyMoE C ABI (include/bfmoe.h): argument checks,
+// workspace layout, tensor maps, launch tracing and the order of the kernels.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "bucket.cuh"
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "materialize.cuh"
+#include "pack.cuh"
+#include "rotate.cuh"
+#include "router.cuh"
+
+using namespace bfmoe;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+int ok() {
+  g_last_error[0] = '\0';
+  return BFMOE_OK;
+}
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(BFMOE_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool is_pow2(long long v) { return v > 0 && (v & (v - 1)) == 0; }
+int ilog2(int v) {
+  int l = 0;
+  while ((1 << l) < v) ++l;
+  return l;
+}
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int words_per_row(int d) { return std::max(1, (d + 15) / 16); }
+
+// ---------------------------------------------------------------------------
+// Launch accounting and optional per-launch CUDA events.
+// ---------------------------------------------------------------------------
+std::atomic<unsigned long long> g_launches{0};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+template <typename F>
+cudaError_t launch(const char* name, cudaStream_t s, F&& f) {
+  ProfRec rec{name, nullptr, nullptr};
+  bool prof;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    prof = g_prof_on;
+    if (prof) {
+      rec.a = pool_event();
+      rec.b = pool_event();
+    }
+  }
+  if (prof) cudaEventRecord(rec.a, s);
+  f();
+  const cudaError_t e = cudaGetLastError();
+  if (prof) {
+    cudaEventRecord(rec.b, s);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.push_back(rec);
+  }
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
+int grid_for(long long work, int per_block, int cap) {
+  long long g = (work + per_block - 1) / per_block;
+  if (g < 1) g = 1;
+  if (g > cap) g = cap;
+  return static_cast<int>(g);
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// ---------------------------------------------------------------------------
+// Workspace: router and forward share one buffer (stream-ordered).
+// ---------------------------------------------------------------------------
+struct Plan {
+  // forward
+  size_t tab_theta, tab_phi, w_bf16, xrot, z, slot, fwd_end;
+  // router
+  size_t logits, chunk_counts, totals, rt_end;
+  size_t total;
+};
+
+Plan make_plan(int d, int N, long long T, int k, int xdt) {
+  Plan p{};
+  const int L = ilog2(d);
+  const long long R = T * k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  const size_t tab = static_cast<size_t>(N) * L * (d / 2) * sizeof(float2);
+  p.tab_theta = take(tab);
+  p.tab_phi = take(tab);
+  p.w_bf16 = take(static_cast<size_t>(d) * d * 2);
+  p.xrot = take(static_cast<size_t>(R) * d * (xdt == BFMOE_BF16 ? 2 : 4));
+  p.z = take(static_cast<size_t>(R) * d * 4);
+  p.slot = take(static_cast<size_t>(R) * d * 4);
+  p.fwd_end = off;
+  off = 0;
+  const long long nchunks = (R + kBucketChunk - 1) / kBucketChunk;
+  p.logits = take(static_cast<size_t>(T) * N * 4);
+  p.chunk_counts = take(static_cast<size_t>(std::max(1LL, nchunks)) * N * 4);
+  p.totals = take(static_cast<size_t>(N) * 4);
+  p.rt_end = off;
+  p.total = std::max(p.fwd_end, p.rt_end);
+  return p;
+}
+
+int check_sizes(int d, int N, long long T, int k) {
+  if (d < 4 || d > BFMOE_MAX_D || !is_pow2(d)) return fail(BFMOE_EINVAL, "d=%d must be a power of two in [4, %d]", d, BFMOE_MAX_D);
+  if (N < 1 || N > BFMOE_MAX_EXPERTS) return fail(BFMOE_EINVAL, "n_experts=%d must be in [1, %d]", N, BFMOE_MAX_EXPERTS);
+  if (k < 1 || k > BFMOE_MAX_K || k > N) return fail(BFMOE_EINVAL, "k=%d must be in [1, min(%d, N=%d)]", k, BFMOE_MAX_K, N);
+  if (T < 0) return fail(BFMOE_EINVAL, "T=%lld must be >= 0", T);
+  if (T * k > 0x7fffffffLL) return fail(BFMOE_EUNSUPPORTED, "T*k=%lld exceeds int32 row ids", T * k);
+  return BFMOE_OK;
+}
+int check_dtype(int xdt) {
+  if (xdt != BFMOE_F32 && xdt != BFMOE_BF16) return fail(BFMOE_EINVAL, "x_dtype=%d is not BFMOE_F32 or BFMOE_BF16", xdt);
+  return BFMOE_OK;
+}
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_ws(const Plan& p, void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return BFMOE_OK;
+  if (!ws) return fail(BFMOE_EWORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(BFMOE_EWORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < need) return fail(BFMOE_EWORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
+  (void)p;
+  return BFMOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor maps (driver entry point looked up through the runtime).
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 [outer][inner], box [box_outer][64] with 128-byte swizzle.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemmBK), box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// Dispatch helpers
+// ---------------------------------------------------------------------------
+template <template <int> class F, typename... A>
+cudaError_t dispatch_e(int d, A&&... a) {
+  switch (d) {
+    case 4: case 8: case 16: case 32: return F<1>::run(std::forward<A>(a)...);
+    case 64: return F<2>::run(std::forward<A>(a)...);
+    case 128: return F<4>::run(std::forward<A>(a)...);
+    case 256: return F<8>::run(std::forward<A>(a)...);
+    case 512: return F<16>::run(std::forward<A>(a)...);
+    case 1024: return F<32>::run(std::forward<A>(a)...);
+    case 2048: return F<64>::run(std::forward<A>(a)...);
+    case 4096: return F<128>::run(std::forward<A>(a)...);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+struct RotArgs {
+  const void* x;
+  bool bf16;
+  const int32_t* idx;
+  const float* gates;
+  const int32_t* rows;
+  const float2* cs;
+  long long R;
+  int k, d, L, N;
+  void* out;
+  const float* z;
+  cudaStream_t s;
+};
+
+template <int E>
+struct PreRotate {
+  static cudaError_t run(const RotArgs& a) {
+    const int grid = grid_for(a.R, 8, sm_count() * 16);
+    return launch("pre_rotate", a.s, [&] {
+      if (a.bf16)
+        pre_rotate_kernel<E, __nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, a.s>>>(
+            static_cast<const __nv_bfloat16*>(a.x), a.idx, a.rows, a.cs, a.R, a.k, a.d, a.L, a.N,
+            static_cast<__nv_bfloat16*>(a.out));
+      else
+        pre_rotate_kernel<E, float, float><<<grid, 256, 0, a.s>>>(static_cast<const float*>(a.x), a.idx, a.rows,
+                                                                   a.cs, a.R, a.k, a.d, a.L, a.N,
+                                                                   static_cast<float*>(a.out));
+    });
+  }
+};
+
+template <int E>
+struct PostRotate {
+  static cudaError_t run(const RotArgs& a) {
+    const int grid = grid_for(a.R, 8, sm_count() * 16);
+    return launch("post_rotate", a.s, [&] {
+      post_rotate_kernel<E><<<grid, 256, 0, a.s>>>(a.z, a.idx, a.gates, a.rows, a.cs, a.R, a.d, a.L, a.N,
+                                                   static_cast<float*>(a.out));
+    });
+  }
+};
+
+template <int BN, int STAGES>
+cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, float* z, int R, int d, float alpha,
+                           cudaStream_t s) {
+  using Cfg = GemmTcCfg<BN, STAGES>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(ternary_gemm_tc_kernel<BN, STAGES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((R + kGemmBM - 1) / kGemmBM, d / BN);
+  return launch("ternary_gemm_tc", s, [&] {
+    ternary_gemm_tc_kernel<BN, STAGES><<<grid, 128, Cfg::SMEM_BYTES, s>>>(ta, tb, z, R, d, alpha);
+  });
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* bfmoe_last_error(void) { return g_last_error; }
+
+unsigned long long bfmoe_launch_count(void) { return g_launches.load(); }
+
+size_t bfmoe_workspace_size(int d, int n_experts, int T, int k, int x_dtype) {
+  if (check_sizes(d, n_experts, T, k) != BFMOE_OK || check_dtype(x_dtype) != BFMOE_OK) return 0;
+  return make_plan(d, n_experts, T, k, x_dtype).total;
+}
+
+int bfmoe_pack_base(const int8_t* w, int d, uint32_t* w_packed, bfmoe_stream_t stream) {
+  if (!w || !w_packed) return fail(BFMOE_EINVAL, "pack_base: NULL pointer");
+  if (d < 4 || d > BFMOE_MAX_D || !is_pow2(d)) return fail(BFMOE_EINVAL, "pack_base: bad d=%d", d);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const unsigned zero = 0;
+  cudaError_t e = cudaMemcpyToSymbolAsync(g_not_ternary, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pack_base: reset flag");
+  const int wpr = words_per_row(d);
+  const long long n = static_cast<long long>(d) * wpr;
+  e = launch("pack_base", s, [&] { pack_base_kernel<<<grid_for(n, 256, 4096), 256, 0, s>>>(w, d, wpr, w_packed); });
+  if (e != cudaSuccess) return cuda_fail(e, "pack_base: launch");
+  unsigned bad = 0;
+  e = cudaMemcpyFromSymbolAsync(&bad, g_not_ternary, sizeof(bad), 0, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "pack_base: read flag");
+  if (bad) return fail(BFMOE_ENOT_TERNARY, "pack_base: a weight is outside {-1, 0, +1}");
+  return ok();
+}
+
+int bfmoe_unpack_base(const uint32_t* w_packed, int d, uint16_t* w_bf16, bfmoe_stream_t stream) {
+  if (!w_packed || !w_bf16) return fail(BFMOE_EINVAL, "unpack_base: NULL pointer");
+  if (d < 4 || d > BFMOE_MAX_D || !is_pow2(d)) return fail(BFMOE_EINVAL, "unpack_base: bad d=%d", d);
+  if (!aligned16(w_bf16)) return fail(BFMOE_EINVAL, "unpack_base: output must be 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int wpr = words_per_row(d);
+  const long long n = static_cast<long long>(d) * wpr;
+  cudaError_t e = launch("expand_base_bf16", s, [&] {
+    expand_base_bf16_kernel<<<grid_for(n, 256, 4096), 256, 0, s>>>(w_packed, d, wpr, w_bf16);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "unpack_base: launch");
+  return ok();
+}
+
+int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_gate, const float* bias,
+                      int n_experts, int k, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets,
+                      int32_t* rows, void* ws, size_t ws_bytes, bfmoe_stream_t stream) {
+  int rc = check_sizes(d, n_experts, T, k);
+  if (rc) return rc;
+  if ((rc = check_dtype(x_dtype))) return rc;
+  if (!counts || !offsets) return fail(BFMOE_EINVAL, "router_topk: NULL counts/offsets");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int N = n_experts;
+  cudaError_t e;
+  if (T == 0) {
+    if ((e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * N, s)) != cudaSuccess) return cuda_fail(e, "router_topk: memset");
+    if ((e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (N + 1), s)) != cudaSuccess) return cuda_fail(e, "router_topk: memset");
+    return ok();
+  }
+  if (!x || !w_gate || !idx || !gates || !rows) return fail(BFMOE_EINVAL, "router_topk: NULL pointer");
+  const Plan p = make_plan(d, N, T, k, x_dtype);
+  if ((rc = check_ws(p, ws, ws_bytes, p.rt_end))) return rc;
+  uint8_t* W = static_cast<uint8_t*>(ws);
+  float* logits = reinterpret_cast<float*>(W + p.logits);
+  int32_t* cc = reinterpret_cast<int32_t*>(W + p.chunk_counts);
+  int32_t* totals = reinterpret_cast<int32_t*>(W + p.totals);
+  const long long R = static_cast<long long>(T) * k;
+
+  dim3 g1((T + 63) / 64, (N + 63) / 64);
+  e = launch("router_logits_simt", s, [&] {
+    if (x_dtype == BFMOE_BF16)
+      router_logits_simt_kernel<__nv_bfloat16><<<g1, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), w_gate,
+                                                                  bias, T, d, N, logits);
+    else
+      router_logits_simt_kernel<float><<<g1, 256, 0, s>>>(static_cast<const float*>(x), w_gate, bias, T, d, N,
+                                                          logits);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "router_topk: logits");
+  e = launch("router_topk", s, [&] {
+    router_topk_kernel<<<grid_for(T, 8, sm_count() * 32), 256, 0, s>>>(logits, T, N, k, idx, gates);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "router_topk: top-k");
+
+  const int nchunks = static_cast<int>((R + kBucketChunk - 1) / kBucketChunk);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(bucket_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BFMOE_MAX_EXPERTS * 4);
+    cudaFuncSetAttribute(bucket_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BFMOE_MAX_EXPERTS * 32);
+    attr = true;
+  }
+  e = launch("bucket_count", s, [&] { bucket_count_kernel<<<nchunks, 1024, N * 4, s>>>(idx, R, N, cc); });
+  if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket count");
+  e = launch("bucket_scan", s, [&] { bucket_scan_kernel<<<(N + 31) / 32, 1024, 0, s>>>(cc, nchunks, N, totals); });
+  if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scan");
+  e = launch("bucket_offsets", s, [&] { bucket_offsets_kernel<<<1, 1024, 0, s>>>(totals, N, counts, offsets); });
+  if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket offsets");
+  e = launch("bucket_scatter", s, [&] {
+    bucket_scatter_kernel<<<nchunks, 1024, N * 32, s>>>(idx, R, N, cc, offsets, rows);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scatter");
+  return ok();
+}
+
+int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, int k, const int32_t* idx,
+                  const float* gates, const int32_t* offsets, const int32_t* rows, void* y, void* ws,
+                  size_t ws_bytes, bfmoe_stream_t stream) {
+  if (!layer) return fail(BFMOE_EINVAL, "forward: NULL layer");
+  const int d = layer->d, N = layer->n_experts;
+  int rc = check_sizes(d, N, T, k);
+  if (rc) return rc;
+  if ((rc = check_dtype(x_dtype))) return rc;
+  if (T == 0) return ok();
+  if (!layer->w_packed || !layer->theta || !layer->phi) return fail(BFMOE_EINVAL, "forward: NULL layer weights");
+  if (!x || !idx || !gates || !offsets || !rows || !y) return fail(BFMOE_EINVAL, "forward: NULL pointer");
+  if (!aligned16(x) || !aligned16(y)) return fail(BFMOE_EINVAL, "forward: x and y must be 16-byte aligned");
+  const Plan p = make_plan(d, N, T, k, x_dtype);
+  if ((rc = check_ws(p, ws, ws_bytes, p.fwd_end))) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* W = static_cast<uint8_t*>(ws);
+  float2* tab_t = reinterpret_cast<float2*>(W + p.tab_theta);
+  float2* tab_p = reinterpret_cast<float2*>(W + p.tab_phi);
+  uint16_t* wbf = reinterpret_cast<uint16_t*>(W + p.w_bf16);
+  void* xrot = W + p.xrot;
+  float* z = reinterpret_cast<float*>(W + p.z);
+  float* slot = reinterpret_cast<float*>(W + p.slot);
+  const int L = ilog2(d);
+  const long long R = static_cast<long long>(T) * k;
+  const bool bf16 = x_dtype == BFMOE_BF16;
+  const int wpr = words_per_row(d);
+  cudaError_t e;
+
+  const long long nang = static_cast<long long>(N) * L * (d / 2);
+  e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->theta, nang, tab_t); });
+  if (e != cudaSuccess) return cuda_fail(e, "forward: theta table");
+  e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->phi, nang, tab_p); });
+  if (e != cudaSuccess) return cuda_fail(e, "forward: phi table");
+
+  RotArgs ra{x, bf16, idx, gates, rows, tab_t, R, k, d, L, N, xrot, nullptr, s};
+  if ((e = dispatch_e<PreRotate>(d, ra)) != cudaSuccess) return cuda_fail(e, "forward: pre-rotation");
+
+  if (bf16 && d >= 64) {
+    const long long nw = static_cast<long long>(d) * wpr;
+    e = launch("expand_base_bf16", s, [&] {
+      expand_base_bf16_kernel<<<grid_for(nw, 256, 4096), 256, 0, s>>>(layer->w_packed, d, wpr, wbf);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "forward: expand base");
+    CUtensorMap ta, tb;
+    const int BN = std::min(d, 256);
+    if (!make_tmap_bf16(&ta, xrot, d, R, kGemmBM) || !make_tmap_bf16(&tb, wbf, d, d, BN))
+      return fail(BFMOE_ECUDA, "forward: tensor map encoding failed");
+    switch (BN) {
+      case 64: e = launch_gemm_tc<64, 4>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
+      case 128: e = launch_gemm_tc<128, 3>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
+      default: e = launch_gemm_tc<256, 2>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "forward: tensor-core GEMM");
+  } else {
+    dim3 g((R + 63) / 64, (d + 63) / 64);
+    e = launch("ternary_gemm_simt", s, [&] {
+      if (bf16)
+        ternary_gemm_simt_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(xrot),
+                                                                  layer->w_packed, wpr, R, d, layer->alpha, z);
+      else
+        ternary_gemm_simt_kernel<float><<<g, 256, 0, s>>>(static_cast<const float*>(xrot), layer->w_packed, wpr, R,
+                                                          d, layer->alpha, z);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "forward: SIMT ternary product");
+  }
+
+  RotArgs rb{nullptr, bf16, idx, gates, rows, tab_p, R, k, d, L, N, slot, z, s};
+  if ((e = dispatch_e<PostRotate>(d, rb)) != cudaSuccess) return cuda_fail(e, "forward: post-rotation");
+
+  const long long n4 = static_cast<long long>(T) * (d / 4);
+  e = launch("combine", s, [&] {
+    if (bf16)
+      combine_kernel<__nv_bfloat16><<<grid_for(n4, 256, sm_count() * 16), 256, 0, s>>>(slot, T, k, d,
+                                                                                      static_cast<__nv_bfloat16*>(y));
+    else
+      combine_kernel<float><<<grid_for(n4, 256, sm_count() * 16), 256, 0, s>>>(slot, T, k, d, static_cast<float*>(y));
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "forward: combine");
+  return ok();
+}
+
+int bfmoe_materialize_expert(const bfmoe_layer* layer, int e_idx, float* w_out, bfmoe_stream_t stream) {
+  if (!layer || !w_out) return fail(BFMOE_EINVAL, "materialize: NULL pointer");
+  const int d = layer->d, N = layer->n_experts;
+  if (d < 4 || d > BFMOE_MAX_D || !is_pow2(d)) return fail(BFMOE_EINVAL, "materialize: bad d=%d", d);
+  if (e_idx < 0 || e_idx >= N) return fail(BFMOE_EINVAL, "materialize: expert %d not in [0, %d)", e_idx, N);
+  if (!layer->w_packed || !layer->theta || !layer->phi) return fail(BFMOE_EINVAL, "materialize: NULL layer weights");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int L = ilog2(d);
+  const size_t per = static_cast<size_t>(L) * (d / 2);
+  cudaError_t e = launch("materialize", s, [&] {
+    materialize_kernel<<<d, 256, 2 * d * sizeof(float), s>>>(layer->w_packed, words_per_row(d), d, L, layer->alpha,
+                                                             layer->theta + per * e_idx, layer->phi + per * e_idx,
+                                                             w_out);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "materialize: launch");
+  return ok();
+}
+
+int bfmoe_check_device_error(bfmoe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "check_device_error: synchronize");
+  unsigned code = 0, info = 0;
+  if ((e = cudaMemcpyFromSymbol(&code, g_err_code, sizeof(code))) != cudaSuccess) return cuda_fail(e, "read error word");
+  if ((e = cudaMemcpyFromSymbol(&info, g_err_info, sizeof(info))) != cudaSuccess) return cuda_fail(e, "read error word");
+  if (code == 0) return ok();
+  const unsigned zero = 0;
+  cudaMemcpyToSymbol(g_err_code, &zero, sizeof(zero));
+  cudaMemcpyToSymbol(g_err_info, &zero, sizeof(zero));
+  if (code == BFMOE_EDEVICE_TIMEOUT) return fail(BFMOE_EDEVICE_TIMEOUT, "device wait timed out (site 0x%x)", info);
+  return fail(static_cast<int>(code), "device check failed (code %u, at %u)", code, info);
+}
+
+int bfmoe_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof) {
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  g_prof_on = on != 0;
+  return ok();
+}
+
+int bfmoe_profile_collect(bfmoe_kernel_time* out, int max, int* n_out) {
+  std::vector<ProfRec> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    recs.swap(g_prof);
+  }
+  std::map<std::string, std::pair<int, double>> agg;
+  std::vector<std::string> order;
+  int rc = BFMOE_OK;
+  for (auto& r : recs) {
+    cudaError_t e = cudaEventSynchronize(r.b);
+    float ms = 0.f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess) rc = cuda_fail(e, "profile_collect");
+    auto it = agg.find(r.name);
+    if (it == agg.end()) {
+      order.push_back(r.name);
+      agg[r.name] = {1, ms};
+    } else {
+      it->second.first += 1;
+      it->second.second += ms;
+    }
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (auto& r : recs) {
+      g_event_pool.push_back(r.a);
+      g_event_pool.push_back(r.b);
+    }
+  }
+  int n = 0;
+  for (auto& name : order) {
+    if (n >= max) break;
+    std::snprintf(out[n].name, sizeof(out[n].name), "%s", name.c_str());
+    out[n].launches = agg[name].first;
+    out[n].total_ms = agg[name].second;
+    ++n;
+  }
+  if (n_out) *n_out = n;
+  return rc == BFMOE_OK ? ok() : rc;
+}
+
+}  // extern "C"

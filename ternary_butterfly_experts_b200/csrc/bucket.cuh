@@ -1,0 +1,150 @@
+// Token-to-expert buckets: a stable counting sort of the routed rows
+// r = t*k + j by expert.  Within an expert, rows come in ascending r, which is
+// ascending token order because a token's k experts are distinct.
+//
+// Rows are cut into chunks of kBucketChunk (one 1024-thread block each):
+//   count    per-chunk expert histogram
+//   scan     per expert, exclusive prefix over chunks (+ totals)
+//   offsets  exclusive prefix over experts (one block)
+//   scatter  position = offsets[e] + chunk prefix + earlier warps of the
+//            chunk + rank among equal experts inside the warp
+#pragma once
+#include "common.cuh"
+
+namespace bfmoe {
+
+constexpr int kBucketChunk = 1024;
+
+__global__ __launch_bounds__(1024) void bucket_count_kernel(const int32_t* __restrict__ idx, long long R, int N,
+                                                            int32_t* __restrict__ chunk_counts) {
+  extern __shared__ int cnt[];
+  for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const long long r = static_cast<long long>(blockIdx.x) * kBucketChunk + threadIdx.x;
+  if (r < R) {
+    const int e = idx[r];
+    if (e >= 0 && e < N) {
+      atomicAdd(&cnt[e], 1);
+    } else {
+      report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(r));
+    }
+  }
+  __syncthreads();
+  int32_t* dst = chunk_counts + static_cast<size_t>(blockIdx.x) * N;
+  for (int e = threadIdx.x; e < N; e += blockDim.x) dst[e] = cnt[e];
+}
+
+// Block of 32 experts (x) by 32 chunk slices (y).  Rewrites chunk_counts
+// into exclusive prefixes over chunks; totals[e] = rows of expert e.
+__global__ __launch_bounds__(1024) void bucket_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int N,
+                                                           int32_t* __restrict__ totals) {
+  __shared__ int part[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + tx;
+  const int per = (nchunks + 31) / 32;
+  const int c0 = min(ty * per, nchunks), c1 = min(c0 + per, nchunks);
+  int s = 0;
+  if (e < N)
+    for (int c = c0; c < c1; ++c) s += chunk_counts[static_cast<size_t>(c) * N + e];
+  part[ty][tx] = s;
+  __syncthreads();
+  if (ty == 0) {
+    int run = 0;
+    for (int q = 0; q < 32; ++q) {
+      const int tmp = part[q][tx];
+      part[q][tx] = run;
+      run += tmp;
+    }
+    if (e < N) totals[e] = run;
+  }
+  __syncthreads();
+  int run = part[ty][tx];
+  if (e < N)
+    for (int c = c0; c < c1; ++c) {
+      const size_t a = static_cast<size_t>(c) * N + e;
+      const int tmp = chunk_counts[a];
+      chunk_counts[a] = run;
+      run += tmp;
+    }
+}
+
+// One block of 1024 threads, N <= 4096 (4 experts per thread).
+__global__ __launch_bounds__(1024) void bucket_offsets_kernel(const int32_t* __restrict__ totals, int N,
+                                                              int32_t* __restrict__ counts,
+                                                              int32_t* __restrict__ offsets) {
+  __shared__ int warp_sum[32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  int v[4];
+  int local = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int e = tid * 4 + q;
+    v[q] = e < N ? totals[e] : 0;
+    local += v[q];
+  }
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(FULL_MASK, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_sum[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int ws = warp_sum[lane];
+    int inc = ws;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(FULL_MASK, inc, off);
+      if (lane >= off) inc += o;
+    }
+    warp_sum[lane] = inc - ws;  // exclusive
+  }
+  __syncthreads();
+  int run = warp_sum[w] + incl - local;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int e = tid * 4 + q;
+    if (e < N) {
+      offsets[e] = run;
+      counts[e] = v[q];
+    }
+    run += v[q];
+  }
+  if (tid == 1023) offsets[N] = run;
+}
+
+__global__ __launch_bounds__(1024) void bucket_scatter_kernel(const int32_t* __restrict__ idx, long long R, int N,
+                                                              const int32_t* __restrict__ chunk_prefix,
+                                                              const int32_t* __restrict__ offsets,
+                                                              int32_t* __restrict__ rows) {
+  extern __shared__ uint8_t wcnt[];  // [N][32]: rows of expert e in warp w
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int q = tid; q < N * 8; q += blockDim.x) reinterpret_cast<uint32_t*>(wcnt)[q] = 0u;
+  __syncthreads();
+  const long long r = static_cast<long long>(blockIdx.x) * kBucketChunk + tid;
+  int e = -1 - lane;
+  bool valid = false;
+  if (r < R) {
+    const int v = idx[r];
+    if (v >= 0 && v < N) {
+      e = v;
+      valid = true;
+    }
+  }
+  const unsigned peers = __match_any_sync(FULL_MASK, e);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  if (valid && rank == 0) wcnt[e * 32 + w] = static_cast<uint8_t>(__popc(peers));
+  __syncthreads();
+  int before = 0;
+  if (valid && rank == 0)
+    for (int q = 0; q < w; ++q) before += wcnt[e * 32 + q];
+  const int leader = __ffs(peers) - 1;
+  before = __shfl_sync(FULL_MASK, before, leader);
+  if (valid) {
+    const int pos = offsets[e] + chunk_prefix[static_cast<size_t>(blockIdx.x) * N + e] + before + rank;
+    rows[pos] = static_cast<int32_t>(r);
+  }
+}
+
+}  // namespace bfmoe

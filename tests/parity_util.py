@@ -1,0 +1,73 @@
+"""Run the CUDA path through the C ABI and compare it with the oracle.
+
+Comparison rules:
+* routing indices bit-exact, except near-tie tokens (oracle float64 logits of
+  neighbouring ranks within 1e-5), which are counted;
+* buckets bit-exact against the oracle's buckets of the GPU's own routing;
+* gates within 1e-5 of the oracle's softmax over the GPU-selected experts;
+* outputs: per-token relative L2 against the oracle evaluated with the GPU's
+  routing (so near-tie tokens still check the arithmetic), at most 1e-5 on
+  the float32 path and 1e-2 on the bfloat16 path.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import bfmoe_oracle as O
+
+TOL = {"f32": 1e-5, "bf16": 1e-2}
+
+
+def run_cuda(inp, device="cuda", check_errors=True):
+    import torch
+    import ternary_butterfly_experts_b200 as B
+
+    wl = inp.wl
+    layer = B.Layer.from_host(inp.w_base, inp.alpha, inp.theta, inp.phi, device=device)
+    x = inp.x.to(device).contiguous()
+    wg = torch.from_numpy(inp.w_gate).to(device)
+    bias = None if inp.bias is None else torch.from_numpy(inp.bias).to(device)
+    code = B.BFMOE_BF16 if wl.dtype == "bf16" else B.BFMOE_F32
+    ws = B.workspace(wl.d, wl.n_experts, x.shape[0], wl.k, code, device)
+    idx, gates, counts, offsets, rows = B.bfmoe_router_topk(x, wg, bias, wl.k, ws)
+    y = B.bfmoe_forward(layer, x, wl.k, idx, gates, offsets, rows, ws)
+    if check_errors:
+        B.bfmoe_check_device_error()
+    torch.cuda.synchronize()
+    return {
+        "idx": idx.cpu().numpy(), "gates": gates.cpu().numpy().astype(np.float64),
+        "counts": counts.cpu().numpy(), "offsets": offsets.cpu().numpy(), "rows": rows.cpu().numpy(),
+        "y": y.float().cpu().numpy().astype(np.float64), "layer": layer, "x": x,
+    }
+
+
+def compare(inp, gpu, tokens=None, tol=None):
+    """Check the GPU results against the oracle.  With ``tokens`` given, only
+    those tokens are evaluated by the oracle (sampled mode for full sizes).
+    Returns a dict of statistics (near ties, max relative error)."""
+    wl = inp.wl
+    tol = TOL[wl.dtype] if tol is None else tol
+    x = inp.x_f64()
+    sel = np.arange(x.shape[0]) if tokens is None else np.asarray(tokens)
+    xs = x[sel]
+    logits = O.router_logits(xs, inp.w_gate, inp.bias)
+    idx_o, near = O.topk(logits, wl.k)
+    idx_g = gpu["idx"][sel].astype(np.int64)
+    mism = (idx_g != idx_o).any(axis=1)
+    bad = mism & ~near
+    assert not bad.any(), f"{int(bad.sum())} non-tie tokens routed differently, e.g. {np.nonzero(bad)[0][:5]}"
+    g_ref = O.gates_for(logits, idx_g)
+    gerr = np.abs(gpu["gates"][sel] - g_ref).max()
+    assert gerr < 1e-5, f"gate error {gerr}"
+    if tokens is None:
+        c, o, r = O.buckets(gpu["idx"], wl.n_experts)
+        assert np.array_equal(gpu["counts"], c), "bucket counts differ"
+        assert np.array_equal(gpu["offsets"], o), "bucket offsets differ"
+        assert np.array_equal(gpu["rows"], r), "bucket rows differ"
+        y_ref = O.forward(xs, inp.w_base, inp.alpha, inp.theta, inp.phi, idx_g, g_ref)
+    else:
+        y_ref = O.forward_tokens(xs, inp.w_base, inp.alpha, inp.theta, inp.phi, idx_g, g_ref)
+    rel = O.rel_l2_per_token(gpu["y"][sel], y_ref)
+    assert rel.max() <= tol, f"max per-token relative L2 {rel.max():.3e} > {tol} (token {sel[rel.argmax()]})"
+    return {"near_ties": int(near.sum()), "mismatched_near_ties": int(mism.sum()),
+            "max_rel_l2": float(rel.max()), "mean_rel_l2": float(rel.mean()), "gate_err": float(gerr)}

@@ -1,0 +1,63 @@
+"""The C ABI library loads on a machine without a GPU, exports every function
+that include/bfmoe.h declares, and rejects bad arguments on the host before
+touching the device."""
+import ctypes
+
+import pytest
+
+from ternary_butterfly_experts_b200 import build, capi
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return capi.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = capi.header_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in bfmoe.h but not exported"
+        assert n in capi.SIGNATURES, f"{n} has no ctypes signature"
+
+
+def test_workspace_size_host_only(L):
+    a = L.bfmoe_workspace_size(512, 256, 16384, 2, capi.BFMOE_BF16)
+    b = L.bfmoe_workspace_size(512, 256, 16384, 2, capi.BFMOE_F32)
+    assert a > 0 and b > a and a % 256 == 0
+    assert L.bfmoe_workspace_size(500, 256, 16384, 2, 1) == 0      # not a power of two
+    assert L.bfmoe_workspace_size(512, 4, 10, 5, 1) == 0           # k > N
+    assert L.bfmoe_workspace_size(512, 4, 10, 9, 1) == 0           # k > 8
+    assert L.bfmoe_workspace_size(512, 4, 10, 2, 7) == 0           # bad dtype
+    assert L.bfmoe_workspace_size(8192, 4, 10, 2, 1) == 0          # d too large
+
+
+def test_argument_checks_before_any_launch(L):
+    n0 = L.bfmoe_launch_count()
+    assert L.bfmoe_pack_base(None, 64, None, None) == capi.BFMOE_EINVAL
+    assert b"NULL" in L.bfmoe_last_error()
+    assert L.bfmoe_pack_base(ctypes.c_void_p(16), 48, ctypes.c_void_p(16), None) == capi.BFMOE_EINVAL
+    lay = capi.BfmoeLayer(64, 4, 16, ctypes.c_float(0.1), 16, 16)
+    assert L.bfmoe_forward(ctypes.byref(lay), None, 1, 4, 2, None, None, None, None, None, None, 0,
+                           None) == capi.BFMOE_EINVAL
+    assert L.bfmoe_forward(ctypes.byref(lay), 16, 1, 4, 5, 16, 16, 16, 16, 16, None, 0, None) == capi.BFMOE_EINVAL
+    assert L.bfmoe_forward(None, 16, 1, 4, 2, 16, 16, 16, 16, 16, None, 0, None) == capi.BFMOE_EINVAL
+    # a workspace that is missing or too small is reported as such
+    assert L.bfmoe_forward(ctypes.byref(lay), 16, 1, 4, 2, 16, 16, 16, 16, 16, None, 0,
+                           None) == capi.BFMOE_EWORKSPACE
+    assert L.bfmoe_forward(ctypes.byref(lay), 16, 1, 4, 2, 16, 16, 16, 16, 16, 256, 10,
+                           None) == capi.BFMOE_EWORKSPACE
+    assert L.bfmoe_forward(ctypes.byref(lay), 16, 1, 4, 2, 16, 16, 16, 16, 16, 258, 1 << 30,
+                           None) == capi.BFMOE_EWORKSPACE   # misaligned
+    assert L.bfmoe_router_topk(16, 1, 4, 64, 16, None, 4, 0, 16, 16, 16, 16, 16, None, 0,
+                               None) == capi.BFMOE_EINVAL     # k = 0
+    assert L.bfmoe_materialize_expert(ctypes.byref(lay), 4, 16, None) == capi.BFMOE_EINVAL
+    assert L.bfmoe_unpack_base(16, 100, 16, None) == capi.BFMOE_EINVAL
+    assert L.bfmoe_launch_count() == n0
+
+
+def test_binding_names_match_header():
+    import ternary_butterfly_experts_b200 as B
+    for n in capi.header_functions():
+        assert hasattr(B, n), f"binding lacks {n}"
