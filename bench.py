@@ -143,6 +143,10 @@ def kernel_costs(wl, tables_bytes):
         "ternary_gemm_simt": ("alu", 2.0 * R * d * d, "TFLOP/s"),
         # router product on the CUDA cores: 2 T N d flops
         "router_logits_simt": ("alu", 2.0 * T * N * d, "TFLOP/s"),
+        # router on the tensor cores: the algorithmic 2 T N d (it issues 3x
+        # that in bf16 MMAs for the exact split of the float32 gate weights)
+        "router_tc": ("tensor", 2.0 * T * N * d, "TFLOP/s"),
+        "router_split": ("hbm", N * d * 4 + 3 * N * d * 2, "GB/s"),
         # pre-rotation: x rows gathered (R rows) + X_rot written + the theta table
         "pre_rotate": ("hbm", R * d * xb + R * d * xb + tables_bytes, "GB/s"),
         # post-rotation: Z read (fp32) + slots written (fp32) + the phi table
@@ -259,9 +263,12 @@ def run_ours(args, wl):
     if world > 1:
         dist.barrier()
     import ternary_butterfly_experts_b200 as B
+    from ternary_butterfly_experts_b200.shard import max_over_ranks, token_range
 
     peaks, peak_src = load_peaks()
-    inp = W.generate(wl, seed=0)
+    # weak scaling: rank r owns tokens [r*T, (r+1)*T) of a world*T batch
+    a, _ = token_range(wl.tokens * world, rank, world)
+    inp = W.generate(wl, seed=0, tokens=wl.tokens, token_offset=a)
     layer = B.Layer.from_host(inp.w_base, inp.alpha, inp.theta, inp.phi, device=dev)
     wg = torch.from_numpy(inp.w_gate).to(dev)
     bias = None if inp.bias is None else torch.from_numpy(inp.bias).to(dev)
@@ -303,10 +310,7 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms)
     B.bfmoe_check_device_error()
 
     # --- per-kernel device times (same steps again, each launch bracketed) ------
@@ -321,10 +325,7 @@ def run_ours(args, wl):
     for _ in range(2):
         model.forward_host(x_host, y_host)
     e2e_ms = timed(args.steps, lambda: model.forward_host(x_host, y_host))
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e2e_ms)
 
     if rank == 0:
         clk = clocks.summary()

@@ -19,7 +19,9 @@
 #include "materialize.cuh"
 #include "pack.cuh"
 #include "rotate.cuh"
+#include "rotate_fast.cuh"
 #include "router.cuh"
+#include "router_tc.cuh"
 
 using namespace bfmoe;
 
@@ -124,7 +126,7 @@ struct Plan {
   // forward
   size_t tab_theta, tab_phi, w_bf16, xrot, z, slot, fwd_end;
   // router
-  size_t logits, chunk_counts, totals, rt_end;
+  size_t logits, chunk_counts, totals, wg_parts, rt_end;
   size_t total;
 };
 
@@ -151,6 +153,7 @@ Plan make_plan(int d, int N, long long T, int k, int xdt) {
   p.logits = take(static_cast<size_t>(T) * N * 4);
   p.chunk_counts = take(static_cast<size_t>(std::max(1LL, nchunks)) * N * 4);
   p.totals = take(static_cast<size_t>(N) * 4);
+  p.wg_parts = take(static_cast<size_t>(3) * N * d * 2);
   p.rt_end = off;
   p.total = std::max(p.fwd_end, p.rt_end);
   return p;
@@ -268,6 +271,65 @@ struct PostRotate {
   }
 };
 
+template <int E>
+struct PreRotateFast {
+  static cudaError_t run(const RotArgs& a) {
+    using Gm = Geo<E>;
+    const size_t smem = static_cast<size_t>(Gm::WARPS) * Gm::D * sizeof(float);
+    if (smem > 48 * 1024) {
+      cudaFuncSetAttribute(pre_rotate_fast_kernel<E, __nv_bfloat16, __nv_bfloat16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      cudaFuncSetAttribute(pre_rotate_fast_kernel<E, float, float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+    }
+    const long long per = static_cast<long long>(Gm::WARPS) * Gm::G;
+    const int grid = static_cast<int>((a.R + per - 1) / per);
+    const float4* q = reinterpret_cast<const float4*>(a.cs);
+    return launch("pre_rotate", a.s, [&] {
+      if (a.bf16)
+        pre_rotate_fast_kernel<E, __nv_bfloat16, __nv_bfloat16><<<grid, 256, smem, a.s>>>(
+            static_cast<const __nv_bfloat16*>(a.x), a.idx, a.rows, q, a.R, a.k, a.N,
+            static_cast<__nv_bfloat16*>(a.out));
+      else
+        pre_rotate_fast_kernel<E, float, float><<<grid, 256, smem, a.s>>>(static_cast<const float*>(a.x), a.idx,
+                                                                           a.rows, q, a.R, a.k, a.N,
+                                                                           static_cast<float*>(a.out));
+    });
+  }
+};
+
+template <int E>
+struct PostRotateFast {
+  static cudaError_t run(const RotArgs& a) {
+    using Gm = Geo<E>;
+    const size_t smem = static_cast<size_t>(Gm::WARPS) * Gm::D * sizeof(float);
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(post_rotate_fast_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+    const long long per = static_cast<long long>(Gm::WARPS) * Gm::G;
+    const int grid = static_cast<int>((a.R + per - 1) / per);
+    const float4* q = reinterpret_cast<const float4*>(a.cs);
+    return launch("post_rotate", a.s, [&] {
+      post_rotate_fast_kernel<E><<<grid, 256, smem, a.s>>>(a.z, a.idx, a.gates, a.rows, q, a.R, a.N,
+                                                           static_cast<float*>(a.out));
+    });
+  }
+};
+
+template <template <int> class F, typename... A>
+cudaError_t dispatch_fast(int d, A&&... a) {
+  switch (d) {
+    case 64: return F<2>::run(std::forward<A>(a)...);
+    case 128: return F<4>::run(std::forward<A>(a)...);
+    case 256: return F<8>::run(std::forward<A>(a)...);
+    case 512: return F<16>::run(std::forward<A>(a)...);
+    case 1024: return F<32>::run(std::forward<A>(a)...);
+    case 2048: return F<64>::run(std::forward<A>(a)...);
+    case 4096: return F<128>::run(std::forward<A>(a)...);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <int BN, int STAGES>
 cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, float* z, int R, int d, float alpha,
                            cudaStream_t s) {
@@ -279,9 +341,27 @@ cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, float* 
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid((R + kGemmBM - 1) / kGemmBM, d / BN);
+  const long long tiles = static_cast<long long>((R + kGemmBM - 1) / kGemmBM) * (d / BN);
+  const int grid = static_cast<int>(std::min<long long>(tiles, sm_count()));
   return launch("ternary_gemm_tc", s, [&] {
-    ternary_gemm_tc_kernel<BN, STAGES><<<grid, 128, Cfg::SMEM_BYTES, s>>>(ta, tb, z, R, d, alpha);
+    ternary_gemm_tc_kernel<BN, STAGES><<<grid, kGemmThreads, Cfg::SMEM_BYTES, s>>>(ta, tb, z, R, d, alpha);
+  });
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_router_tc(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
+                             int k, int32_t* idx, float* gates, cudaStream_t s) {
+  using Cfg = RouterTcCfg<BN, STAGES>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = (T + kGemmBM - 1) / kGemmBM;
+  return launch("router_tc", s, [&] {
+    router_tc_kernel<BN, STAGES><<<grid, kRouterThreads, Cfg::SMEM_BYTES, s>>>(tx, tw, bias, T, d, N, k, idx, gates);
   });
 }
 
@@ -358,20 +438,40 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
   int32_t* totals = reinterpret_cast<int32_t*>(W + p.totals);
   const long long R = static_cast<long long>(T) * k;
 
-  dim3 g1((T + 63) / 64, (N + 63) / 64);
-  e = launch("router_logits_simt", s, [&] {
-    if (x_dtype == BFMOE_BF16)
-      router_logits_simt_kernel<__nv_bfloat16><<<g1, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), w_gate,
-                                                                  bias, T, d, N, logits);
-    else
-      router_logits_simt_kernel<float><<<g1, 256, 0, s>>>(static_cast<const float*>(x), w_gate, bias, T, d, N,
-                                                          logits);
-  });
-  if (e != cudaSuccess) return cuda_fail(e, "router_topk: logits");
-  e = launch("router_topk", s, [&] {
-    router_topk_kernel<<<grid_for(T, 8, sm_count() * 32), 256, 0, s>>>(logits, T, N, k, idx, gates);
-  });
-  if (e != cudaSuccess) return cuda_fail(e, "router_topk: top-k");
+  if (x_dtype == BFMOE_BF16 && d % kGemmBK == 0) {
+    // tensor cores: exact 3-way bf16 split of W_g, top-k fused in the epilogue
+    if (!aligned16(x)) return fail(BFMOE_EINVAL, "router_topk: x must be 16-byte aligned");
+    __nv_bfloat16* parts = reinterpret_cast<__nv_bfloat16*>(W + p.wg_parts);
+    const long long nw = static_cast<long long>(N) * d;
+    e = launch("router_split", s, [&] { router_split_kernel<<<grid_for(nw, 256, 2048), 256, 0, s>>>(w_gate, nw, parts); });
+    if (e != cudaSuccess) return cuda_fail(e, "router_topk: split");
+    const int BN = N >= 128 ? 128 : (N > 32 ? 64 : (N > 16 ? 32 : 16));
+    CUtensorMap tx, tw;
+    if (!make_tmap_bf16(&tx, x, d, T, kGemmBM) || !make_tmap_bf16(&tw, parts, d, 3LL * N, BN))
+      return fail(BFMOE_ECUDA, "router_topk: tensor map encoding failed");
+    switch (BN) {
+      case 16: e = launch_router_tc<16, 4>(tx, tw, bias, T, d, N, k, idx, gates, s); break;
+      case 32: e = launch_router_tc<32, 4>(tx, tw, bias, T, d, N, k, idx, gates, s); break;
+      case 64: e = launch_router_tc<64, 4>(tx, tw, bias, T, d, N, k, idx, gates, s); break;
+      default: e = launch_router_tc<128, 3>(tx, tw, bias, T, d, N, k, idx, gates, s); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "router_topk: tensor-core router");
+  } else {
+    dim3 g1((T + 63) / 64, (N + 63) / 64);
+    e = launch("router_logits_simt", s, [&] {
+      if (x_dtype == BFMOE_BF16)
+        router_logits_simt_kernel<__nv_bfloat16><<<g1, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), w_gate,
+                                                                    bias, T, d, N, logits);
+      else
+        router_logits_simt_kernel<float><<<g1, 256, 0, s>>>(static_cast<const float*>(x), w_gate, bias, T, d, N,
+                                                            logits);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "router_topk: logits");
+    e = launch("router_topk", s, [&] {
+      router_topk_kernel<<<grid_for(T, 8, sm_count() * 32), 256, 0, s>>>(logits, T, N, k, idx, gates);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "router_topk: top-k");
+  }
 
   const int nchunks = static_cast<int>((R + kBucketChunk - 1) / kBucketChunk);
   static bool attr = false;
@@ -421,14 +521,27 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
   const int wpr = words_per_row(d);
   cudaError_t e;
 
+  const bool fast = d >= 64;
   const long long nang = static_cast<long long>(N) * L * (d / 2);
-  e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->theta, nang, tab_t); });
-  if (e != cudaSuccess) return cuda_fail(e, "forward: theta table");
-  e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->phi, nang, tab_p); });
-  if (e != cudaSuccess) return cuda_fail(e, "forward: phi table");
+  if (fast) {
+    const long long nq = nang / 2;
+    e = launch("rot_table", s, [&] {
+      rot_quads_kernel<<<grid_for(nq, 256, 8192), 256, 0, s>>>(layer->theta, N, d, L, reinterpret_cast<float4*>(tab_t));
+    });
+    if (e == cudaSuccess)
+      e = launch("rot_table", s, [&] {
+        rot_quads_kernel<<<grid_for(nq, 256, 8192), 256, 0, s>>>(layer->phi, N, d, L, reinterpret_cast<float4*>(tab_p));
+      });
+  } else {
+    e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->theta, nang, tab_t); });
+    if (e == cudaSuccess)
+      e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->phi, nang, tab_p); });
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "forward: rotation tables");
 
   RotArgs ra{x, bf16, idx, gates, rows, tab_t, R, k, d, L, N, xrot, nullptr, s};
-  if ((e = dispatch_e<PreRotate>(d, ra)) != cudaSuccess) return cuda_fail(e, "forward: pre-rotation");
+  e = fast ? dispatch_fast<PreRotateFast>(d, ra) : dispatch_e<PreRotate>(d, ra);
+  if (e != cudaSuccess) return cuda_fail(e, "forward: pre-rotation");
 
   if (bf16 && d >= 64) {
     const long long nw = static_cast<long long>(d) * wpr;
@@ -441,9 +554,9 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
     if (!make_tmap_bf16(&ta, xrot, d, R, kGemmBM) || !make_tmap_bf16(&tb, wbf, d, d, BN))
       return fail(BFMOE_ECUDA, "forward: tensor map encoding failed");
     switch (BN) {
-      case 64: e = launch_gemm_tc<64, 4>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
-      case 128: e = launch_gemm_tc<128, 3>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
-      default: e = launch_gemm_tc<256, 2>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
+      case 64: e = launch_gemm_tc<64, 8>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
+      case 128: e = launch_gemm_tc<128, 6>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
+      default: e = launch_gemm_tc<256, 4>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "forward: tensor-core GEMM");
   } else {
@@ -460,7 +573,8 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
   }
 
   RotArgs rb{nullptr, bf16, idx, gates, rows, tab_p, R, k, d, L, N, slot, z, s};
-  if ((e = dispatch_e<PostRotate>(d, rb)) != cudaSuccess) return cuda_fail(e, "forward: post-rotation");
+  e = fast ? dispatch_fast<PostRotateFast>(d, rb) : dispatch_e<PostRotate>(d, rb);
+  if (e != cudaSuccess) return cuda_fail(e, "forward: post-rotation");
 
   const long long n4 = static_cast<long long>(T) * (d / 4);
   e = launch("combine", s, [&] {

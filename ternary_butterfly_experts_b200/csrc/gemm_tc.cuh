@@ -3,13 +3,17 @@
 // the step "ternary multiply with the shared base" of the ButterflyMoE
 // inference (technical summary, 2.3).  Because W_base is shared by every
 // expert, all R routed rows form one dense GEMM; no grouped GEMM is needed.
-// The ternary weights are exact in bf16, the product accumulates in fp32.
+// The ternary weights are exact in bf16; the product accumulates in fp32.
 //
-// Per CTA: one 128 x BN output tile.  Warp 0 (one lane) streams 128x64 A and
-// BNx64 B tiles with TMA (128-byte swizzle) into a STAGES-deep ring; warp 1
-// (one lane) issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM accumulator;
-// all four warps then drain TMEM (warp w owns lanes 32w..32w+31 = rows) and
-// store alpha * acc.
+// Persistent kernel, one CTA per SM, 128 x BN output tiles:
+//   warp 0 (one lane)  TMA producer: 128x64 A and BNx64 B tiles (128-byte
+//                      swizzle) into a STAGES-deep shared-memory ring;
+//   warp 1 (one lane)  MMA issuer: tcgen05.mma M=128 N=BN K=16 into one of two
+//                      TMEM accumulators (2*BN columns);
+//   warps 2..5         epilogue: TMEM -> registers -> alpha * acc -> a per-warp
+//                      shared-memory transpose -> coalesced stores of Z; the
+//                      accumulator is released as soon as it is read, so the
+//                      next tile's MMAs overlap this tile's stores.
 #pragma once
 #include "common.cuh"
 
@@ -17,105 +21,154 @@ namespace bfmoe {
 
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 64;
+constexpr int kGemmThreads = 192;
 
 template <int BN, int STAGES>
 struct GemmTcCfg {
   static constexpr uint32_t A_BYTES = kGemmBM * kGemmBK * 2;
   static constexpr uint32_t B_BYTES = BN * kGemmBK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t BAR_BYTES = (2 * STAGES + 1) * 8 + 8;
-  static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr uint32_t EPI_BYTES = 4 * 32 * 32 * 4;  // 4 warps x 32x32 fp32
+  static constexpr uint32_t BAR_BYTES = (2 * STAGES + 4) * 8 + 8;
+  static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
 };
 
 template <int BN, int STAGES>
-__global__ __launch_bounds__(128, 1) void ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
-                                                                 const __grid_constant__ CUtensorMap tmB,
-                                                                 float* __restrict__ Z, int R, int d, float alpha) {
+__global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+                                                                          const __grid_constant__ CUtensorMap tmB,
+                                                                          float* __restrict__ Z, int R, int d,
+                                                                          float alpha) {
   using Cfg = GemmTcCfg<BN, STAGES>;
-  static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "TMEM columns must be a power of two >= 32");
+  static_assert(2 * BN == 64 || 2 * BN == 128 || 2 * BN == 256 || 2 * BN == 512, "TMEM columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  float* epi = reinterpret_cast<float*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES + Cfg::EPI_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* accb = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accb + 1);
+  uint64_t* tfull = empty + STAGES;  // [2]
+  uint64_t* tempty = tfull + 2;      // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kGemmBM, n0 = blockIdx.y * BN;
   const int nk = d / kGemmBK;
+  const int n_tiles_n = d / BN;
+  const int n_tiles = ((R + kGemmBM - 1) / kGemmBM) * n_tiles_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    mbar_init(accb, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, 4);
+    }
     mbar_fence_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
-  if (warp == 0) tmem_alloc(tmem_slot, BN);
+  if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 && lane == 0) {
-    // TMA producer
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1u;
-      if (kb >= STAGES && !mbar_wait(empty + s, ph ^ 1u, 0x100u | s)) break;
-      mbar_expect_tx(full + s, Cfg::STAGE_BYTES);
-      uint8_t* a = smem + s * Cfg::STAGE_BYTES;
-      tma_load_2d(a, &tmA, full + s, kb * kGemmBK, m0);
-      tma_load_2d(a + Cfg::A_BYTES, &tmB, full + s, kb * kGemmBK, n0);
-    }
-  } else if (warp == 1 && lane == 0) {
-    // MMA issuer
-    constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, BN);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1u;
-      if (!mbar_wait(full + s, ph, 0x200u | s)) break;
-      tc_fence_after();
-      const uint32_t a = smem_u32(smem + s * Cfg::STAGE_BYTES);
-      const uint64_t ad = desc_kmajor_sw128(a);
-      const uint64_t bd = desc_kmajor_sw128(a + Cfg::A_BYTES);
-#pragma unroll
-      for (int kk = 0; kk < kGemmBK / 16; ++kk) {
-        // +32 bytes along K inside the 128-byte swizzle atom = +2 in the
-        // descriptor's 16-byte address units.
-        mma_bf16_ss(tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+        const int m0 = (t / n_tiles_n) * kGemmBM, n0 = (t % n_tiles_n) * BN;
+        bool alive = true;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (it >= STAGES && !mbar_wait(empty + s, ph ^ 1u, 0x100u | s)) {
+            alive = false;
+            break;
+          }
+          mbar_expect_tx(full + s, Cfg::STAGE_BYTES);
+          uint8_t* a = smem + s * Cfg::STAGE_BYTES;
+          tma_load_2d(a, &tmA, full + s, kb * kGemmBK, m0);
+          tma_load_2d(a + Cfg::A_BYTES, &tmB, full + s, kb * kGemmBK, n0);
+        }
+        if (!alive) break;
       }
-      mma_commit(empty + s);
     }
-    mma_commit(accb);
-  }
-  __syncwarp();
-
-  // Epilogue: TMEM -> registers -> global.
-  const bool ok = mbar_wait(accb, 0, 0x300u);
-  tc_fence_after();
-  const int row = m0 + warp * 32 + lane;
-  if (ok) {
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c), v);
-      tmem_wait_ld();
-      if (row < R) {
-        float4* dst = reinterpret_cast<float4*>(Z + static_cast<size_t>(row) * d + n0 + c);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, BN);
+      int it = 0, i = 0;
+      bool alive = true;
+      for (int t = blockIdx.x; t < n_tiles && alive; t += gridDim.x, ++i) {
+        const int buf = i & 1;
+        if (i >= 2 && !mbar_wait(tempty + buf, ((i >> 1) - 1) & 1u, 0x300u | buf)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * BN);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(full + s, ph, 0x200u | s)) {
+            alive = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + s * Cfg::STAGE_BYTES);
+          const uint64_t ad = desc_kmajor_sw128(a);
+          const uint64_t bd = desc_kmajor_sw128(a + Cfg::A_BYTES);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          dst[q] = make_float4(alpha * __uint_as_float(v[4 * q]), alpha * __uint_as_float(v[4 * q + 1]),
-                               alpha * __uint_as_float(v[4 * q + 2]), alpha * __uint_as_float(v[4 * q + 3]));
+          for (int kk = 0; kk < kGemmBK / 16; ++kk)
+            mma_bf16_ss(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          mma_commit(empty + s);
+        }
+        mma_commit(tfull + buf);
+      }
+    }
+  } else {
+    // epilogue warps 2..5: TMEM sub-partition (warp % 4) holds rows 32*(warp%4) ..
+    const int sp = warp & 3;
+    float* buf_w = epi + (warp - 2) * 32 * 32;
+    int i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+      const int m0 = (t / n_tiles_n) * kGemmBM, n0 = (t % n_tiles_n) * BN;
+      const int buf = i & 1;
+      if (!mbar_wait(tfull + buf, (i >> 1) & 1u, 0x400u | buf)) break;
+      tc_fence_after();
+      const uint32_t base = tmem + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(buf * BN);
+      const int row0 = m0 + sp * 32;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(base + static_cast<uint32_t>(c), v);
+        tmem_wait_ld();
+        if (c + 32 >= BN) {
+          // whole accumulator read: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty + buf);
+        }
+        // lane = row: write 8 float4 (swizzled by row) ...
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<float4*>(buf_w + lane * 32 + ((u ^ (lane & 7)) << 2)) =
+              make_float4(alpha * __uint_as_float(v[4 * u]), alpha * __uint_as_float(v[4 * u + 1]),
+                          alpha * __uint_as_float(v[4 * u + 2]), alpha * __uint_as_float(v[4 * u + 3]));
+        __syncwarp();
+        // ... then 4 rows x 128 bytes per store instruction
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int rr = q * 4 + (lane >> 3), u = lane & 7;
+          const float4 val = *reinterpret_cast<const float4*>(buf_w + rr * 32 + ((u ^ (rr & 7)) << 2));
+          const int row = row0 + rr;
+          if (row < R) *reinterpret_cast<float4*>(Z + static_cast<size_t>(row) * d + n0 + c + 4 * u) = val;
+        }
+        __syncwarp();
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, BN);
+  if (warp == 0) tmem_dealloc(tmem, Cfg::TMEM_COLS);
 }
 
 }  // namespace bfmoe

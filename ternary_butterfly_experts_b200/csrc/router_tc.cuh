@@ -1,0 +1,226 @@
+// Router on the tensor cores, with top-k and gates fused into the epilogue.
+//
+// logits = x W_g^T + b with x in bfloat16 and W_g in float32.  W_g is split
+// exactly into three bfloat16 parts, w = hi + mid + lo (each part holds the
+// next 8 significant bits; the remainders are exact in float32), so the
+// logits are three bf16 x bf16 products with exact terms, accumulated in
+// float32 in tensor memory: the same sum as a float32 dot product, in another
+// order.
+//
+// One CTA owns 128 tokens and walks the experts in chunks of BN columns.
+// Warp 0 (one lane) loads with TMA the 128x64 token tile and the three BNx64
+// weight tiles per 64-wide slice of d; warp 1 (one lane) issues the MMAs into
+// one of two TMEM accumulators; warps 2..5 read their rows' logits from TMEM
+// (warp w owns TMEM lanes 32*(w%4) ..), keep a running top-k (larger logit
+// first, lower expert index on ties, NaN below every number) while the next
+// chunk is being multiplied, and finally write idx and the renormalised
+// gates.
+#pragma once
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "router.cuh"
+
+namespace bfmoe {
+
+// w [N][d] float32 -> parts [3][N][d] bfloat16 with hi + mid + lo == w.
+__global__ void router_split_kernel(const float* __restrict__ w, long long n, __nv_bfloat16* __restrict__ parts) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float v = w[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    parts[i] = hi;
+    parts[n + i] = mid;
+    parts[2 * n + i] = __float2bfloat16_rn(r2);
+  }
+}
+
+template <int BN, int STAGES>
+struct RouterTcCfg {
+  static constexpr uint32_t A_BYTES = kGemmBM * kGemmBK * 2;
+  static constexpr uint32_t B_BYTES = BN * kGemmBK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + 3 * B_BYTES;
+  static constexpr uint32_t BAR_BYTES = (2 * STAGES + 4) * 8 + 8;
+  static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : 256));
+};
+
+constexpr int kRouterThreads = 192;
+
+template <int BN, int STAGES>
+__global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                                                           const __grid_constant__ CUtensorMap tmW,
+                                                           const float* __restrict__ bias, int T, int d, int N,
+                                                           int k, int32_t* __restrict__ idx,
+                                                           float* __restrict__ gates) {
+  using Cfg = RouterTcCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kGemmBM;
+  const int nk = d / kGemmBK;
+  const int nchunks = (N + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full + b, 1);
+      mbar_init(acc_empty + b, 4);  // one arrival per epilogue warp
+    }
+    mbar_fence_init();
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    int it = 0;
+    bool alive = true;
+    for (int c = 0; c < nchunks && alive; ++c) {
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        if (it >= STAGES && !mbar_wait(empty + s, ph ^ 1u, 0x1100u | s)) {
+          alive = false;
+          break;
+        }
+        mbar_expect_tx(full + s, Cfg::STAGE_BYTES);
+        uint8_t* a = smem + s * Cfg::STAGE_BYTES;
+        tma_load_2d(a, &tmX, full + s, kb * kGemmBK, m0);
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+          tma_load_2d(a + Cfg::A_BYTES + p * Cfg::B_BYTES, &tmW, full + s, kb * kGemmBK, p * N + c * BN);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, BN);
+    int it = 0;
+    bool alive = true;
+    for (int c = 0; c < nchunks && alive; ++c) {
+      const int buf = c & 1;
+      if (c >= 2 && !mbar_wait(acc_empty + buf, ((c >> 1) - 1) & 1u, 0x1300u | buf)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * BN);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        if (!mbar_wait(full + s, ph, 0x1200u | s)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + s * Cfg::STAGE_BYTES);
+        const uint64_t ad = desc_kmajor_sw128(a);
+#pragma unroll
+        for (int p = 0; p < 3; ++p) {
+          const uint64_t bd = desc_kmajor_sw128(a + Cfg::A_BYTES + p * Cfg::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; ++kk)
+            mma_bf16_ss(d_tmem, ad + 2u * kk, bd + 2u * kk, idesc, (kb | kk | p) != 0 ? 1u : 0u);
+        }
+        mma_commit(empty + s);
+      }
+      mma_commit(acc_full + buf);
+    }
+  }
+  if (warp < 2) {
+    // producer and MMA warps take no part in the epilogue
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+    return;
+  }
+
+  // Epilogue (warps 2..5): one token row per thread.
+  const int sp = warp & 3;
+  const int row = m0 + sp * 32 + lane;
+  float v[BFMOE_MAX_K];
+  int id[BFMOE_MAX_K];
+#pragma unroll
+  for (int j = 0; j < BFMOE_MAX_K; ++j) {
+    v[j] = -INFINITY;
+    id[j] = 0x7fffffff;
+  }
+  float th_v = -INFINITY;
+  int th_i = 0x7fffffff;
+  bool ok = true;
+  for (int c = 0; c < nchunks; ++c) {
+    const int buf = c & 1;
+    if (!mbar_wait(acc_full + buf, (c >> 1) & 1u, 0x1400u | buf)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    const uint32_t base = tmem + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(buf * BN);
+#pragma unroll 1
+    for (int col = 0; col < BN; col += 32) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(base + static_cast<uint32_t>(col), r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const int e = c * BN + col + q;
+        if (e >= N) break;
+        float l = __uint_as_float(r[q]) + (bias ? __ldg(bias + e) : 0.f);
+        if (isnan(l)) l = -INFINITY;
+        if (!ranks_before(l, e, th_v, th_i)) continue;
+        float cv = l;
+        int ci = e;
+#pragma unroll
+        for (int j = 0; j < BFMOE_MAX_K; ++j) {
+          if (j < k && ranks_before(cv, ci, v[j], id[j])) {
+            const float tv = v[j];
+            const int ti = id[j];
+            v[j] = cv;
+            id[j] = ci;
+            cv = tv;
+            ci = ti;
+          }
+          if (j == k - 1) {
+            th_v = v[j];
+            th_i = id[j];
+          }
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acc_empty + buf);
+  }
+  if (ok && row < T) {
+    float z[BFMOE_MAX_K];
+    float sum = 0.f;
+    const bool finite_top = v[0] > -INFINITY;
+#pragma unroll
+    for (int j = 0; j < BFMOE_MAX_K; ++j) {
+      if (j >= k) break;
+      z[j] = finite_top ? expf(v[j] - v[0]) : 1.f;
+      sum += z[j];
+    }
+#pragma unroll
+    for (int j = 0; j < BFMOE_MAX_K; ++j) {
+      if (j >= k) break;
+      idx[static_cast<size_t>(row) * k + j] = id[j];
+      gates[static_cast<size_t>(row) * k + j] = z[j] / sum;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+}
+
+}  // namespace bfmoe

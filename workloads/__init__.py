@@ -106,8 +106,11 @@ class Inputs:
         return self.x.float().double().numpy()
 
 
-def generate(wl: Workload, seed: int = 0, tokens: Optional[int] = None) -> Inputs:
-    """Draw the inputs of ``wl`` (see the module docstring for the recipe)."""
+def generate(wl: Workload, seed: int = 0, tokens: Optional[int] = None, token_offset: int = 0) -> Inputs:
+    """Draw the inputs of ``wl`` (see the module docstring for the recipe).
+
+    ``token_offset`` returns rows [token_offset, token_offset + tokens) of a
+    longer token draw (one shard of a larger batch, same weights)."""
     import torch
 
     d, n = wl.d, wl.n_experts
@@ -130,7 +133,7 @@ def generate(wl: Workload, seed: int = 0, tokens: Optional[int] = None) -> Input
     n_out = int(round(wl.outlier_frac * d))
     outliers = (rng.choice(d, size=n_out, replace=False) if n_out > 0
                 else np.zeros((0,), dtype=np.int64))
-    x = rng.normal(0.0, 1.0, size=(T, d))
+    x = rng.normal(0.0, 1.0, size=(token_offset + T, d))[token_offset:]
     if n_out > 0:
         x[:, outliers] *= wl.outlier_scale
     xt = torch.from_numpy(x.astype(np.float32))
