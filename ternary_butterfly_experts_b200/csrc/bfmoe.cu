@@ -140,13 +140,17 @@ Plan make_plan(int d, int N, long long T, int k, int xdt) {
     off += align_up(bytes, 256);
     return o;
   };
-  const size_t tab = static_cast<size_t>(N) * L * (d / 2) * sizeof(float2);
-  p.tab_theta = take(tab);
-  p.tab_phi = take(tab);
+  // cos/sin tables: theta then phi (quad layout for d >= 64, (c, s) pairs below)
+  const size_t tab = d >= 64 ? static_cast<size_t>(N) * tab_quads(d / 32) * sizeof(float4)
+                             : static_cast<size_t>(N) * L * (d / 2) * sizeof(float2);
+  p.tab_theta = take(2 * tab);
+  p.tab_phi = p.tab_theta + tab;
   p.w_bf16 = take(static_cast<size_t>(d) * d * 2);
   p.xrot = take(static_cast<size_t>(R) * d * (xdt == BFMOE_BF16 ? 2 : 4));
-  p.z = take(static_cast<size_t>(R) * d * 4);
-  p.slot = take(static_cast<size_t>(R) * d * 4);
+  // the bf16 tensor-core path keeps Z and the per-slot outputs in bf16
+  const size_t inter = (xdt == BFMOE_BF16 && d >= 64) ? 2 : 4;
+  p.z = take(static_cast<size_t>(R) * d * inter);
+  p.slot = take(static_cast<size_t>(R) * d * inter);
   p.fwd_end = off;
   off = 0;
   const long long nchunks = (R + kBucketChunk - 1) / kBucketChunk;
@@ -239,7 +243,7 @@ struct RotArgs {
   long long R;
   int k, d, L, N;
   void* out;
-  const float* z;
+  const void* z;
   cudaStream_t s;
 };
 
@@ -265,8 +269,8 @@ struct PostRotate {
   static cudaError_t run(const RotArgs& a) {
     const int grid = grid_for(a.R, 8, sm_count() * 16);
     return launch("post_rotate", a.s, [&] {
-      post_rotate_kernel<E><<<grid, 256, 0, a.s>>>(a.z, a.idx, a.gates, a.rows, a.cs, a.R, a.d, a.L, a.N,
-                                                   static_cast<float*>(a.out));
+      post_rotate_kernel<E><<<grid, 256, 0, a.s>>>(static_cast<const float*>(a.z), a.idx, a.gates, a.rows, a.cs,
+                                                   a.R, a.d, a.L, a.N, static_cast<float*>(a.out));
     });
   }
 };
@@ -274,46 +278,50 @@ struct PostRotate {
 template <int E>
 struct PreRotateFast {
   static cudaError_t run(const RotArgs& a) {
-    using Gm = Geo<E>;
-    const size_t smem = static_cast<size_t>(Gm::WARPS) * Gm::D * sizeof(float);
-    if (smem > 48 * 1024) {
+    using Cb = StagedCfg<E, __nv_bfloat16>;
+    using Cf = StagedCfg<E, float>;
+    static bool attr = false;
+    if (!attr) {
       cudaFuncSetAttribute(pre_rotate_fast_kernel<E, __nv_bfloat16, __nv_bfloat16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cb::SMEM));
       cudaFuncSetAttribute(pre_rotate_fast_kernel<E, float, float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
+                           static_cast<int>(Cf::SMEM));
+      attr = true;
     }
-    const long long per = static_cast<long long>(Gm::WARPS) * Gm::G;
-    const int grid = static_cast<int>((a.R + per - 1) / per);
     const float4* q = reinterpret_cast<const float4*>(a.cs);
     return launch("pre_rotate", a.s, [&] {
       if (a.bf16)
-        pre_rotate_fast_kernel<E, __nv_bfloat16, __nv_bfloat16><<<grid, 256, smem, a.s>>>(
-            static_cast<const __nv_bfloat16*>(a.x), a.idx, a.rows, q, a.R, a.k, a.N,
-            static_cast<__nv_bfloat16*>(a.out));
+        pre_rotate_fast_kernel<E, __nv_bfloat16, __nv_bfloat16>
+            <<<static_cast<int>((a.R + Cb::ROWS - 1) / Cb::ROWS), Cb::THREADS, Cb::SMEM, a.s>>>(
+                static_cast<const __nv_bfloat16*>(a.x), a.idx, a.rows, q, a.R, a.k, a.N,
+                static_cast<__nv_bfloat16*>(a.out));
       else
-        pre_rotate_fast_kernel<E, float, float><<<grid, 256, smem, a.s>>>(static_cast<const float*>(a.x), a.idx,
-                                                                           a.rows, q, a.R, a.k, a.N,
-                                                                           static_cast<float*>(a.out));
+        pre_rotate_fast_kernel<E, float, float>
+            <<<static_cast<int>((a.R + Cf::ROWS - 1) / Cf::ROWS), Cf::THREADS, Cf::SMEM, a.s>>>(
+                static_cast<const float*>(a.x), a.idx, a.rows, q, a.R, a.k, a.N, static_cast<float*>(a.out));
     });
   }
 };
 
 template <int E>
 struct PostRotateFast {
-  static cudaError_t run(const RotArgs& a) {
-    using Gm = Geo<E>;
-    const size_t smem = static_cast<size_t>(Gm::WARPS) * Gm::D * sizeof(float);
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(post_rotate_fast_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
-    const long long per = static_cast<long long>(Gm::WARPS) * Gm::G;
-    const int grid = static_cast<int>((a.R + per - 1) / per);
+  template <typename T>
+  static cudaError_t go(const RotArgs& a) {
+    using C = StagedCfg<E, T>;
+    static bool attr = false;
+    if (!attr) {
+      cudaFuncSetAttribute(post_rotate_fast_kernel<E, T, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(C::SMEM));
+      attr = true;
+    }
     const float4* q = reinterpret_cast<const float4*>(a.cs);
     return launch("post_rotate", a.s, [&] {
-      post_rotate_fast_kernel<E><<<grid, 256, smem, a.s>>>(a.z, a.idx, a.gates, a.rows, q, a.R, a.N,
-                                                           static_cast<float*>(a.out));
+      post_rotate_fast_kernel<E, T, T><<<static_cast<int>((a.R + C::ROWS - 1) / C::ROWS), C::THREADS, C::SMEM, a.s>>>(
+          static_cast<const T*>(a.z), a.idx, a.gates, a.rows, q, a.R, a.N, static_cast<T*>(a.out));
     });
   }
+  // bf16 path: Z and slots in bf16; float32 path: float32
+  static cudaError_t run(const RotArgs& a) { return a.bf16 ? go<__nv_bfloat16>(a) : go<float>(a); }
 };
 
 template <template <int> class F, typename... A>
@@ -331,7 +339,7 @@ cudaError_t dispatch_fast(int d, A&&... a) {
 }
 
 template <int BN, int STAGES>
-cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, float* z, int R, int d, float alpha,
+cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, __nv_bfloat16* z, int R, int d, float alpha,
                            cudaStream_t s) {
   using Cfg = GemmTcCfg<BN, STAGES>;
   static bool attr = false;
@@ -348,21 +356,36 @@ cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, float* 
   });
 }
 
-template <int BN, int STAGES>
-cudaError_t launch_router_tc(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
-                             int k, int32_t* idx, float* gates, cudaStream_t s) {
+template <int BN, int STAGES, int K>
+cudaError_t launch_router_tc_k(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
+                               int32_t* idx, float* gates, cudaStream_t s) {
   using Cfg = RouterTcCfg<BN, STAGES>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<BN, STAGES, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int grid = (T + kGemmBM - 1) / kGemmBM;
   return launch("router_tc", s, [&] {
-    router_tc_kernel<BN, STAGES><<<grid, kRouterThreads, Cfg::SMEM_BYTES, s>>>(tx, tw, bias, T, d, N, k, idx, gates);
+    router_tc_kernel<BN, STAGES, K><<<grid, kRouterThreads, Cfg::SMEM_BYTES, s>>>(tx, tw, bias, T, d, N, idx, gates);
   });
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_router_tc(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
+                             int k, int32_t* idx, float* gates, cudaStream_t s) {
+  switch (k) {
+    case 1: return launch_router_tc_k<BN, STAGES, 1>(tx, tw, bias, T, d, N, idx, gates, s);
+    case 2: return launch_router_tc_k<BN, STAGES, 2>(tx, tw, bias, T, d, N, idx, gates, s);
+    case 3: return launch_router_tc_k<BN, STAGES, 3>(tx, tw, bias, T, d, N, idx, gates, s);
+    case 4: return launch_router_tc_k<BN, STAGES, 4>(tx, tw, bias, T, d, N, idx, gates, s);
+    case 5: return launch_router_tc_k<BN, STAGES, 5>(tx, tw, bias, T, d, N, idx, gates, s);
+    case 6: return launch_router_tc_k<BN, STAGES, 6>(tx, tw, bias, T, d, N, idx, gates, s);
+    case 7: return launch_router_tc_k<BN, STAGES, 7>(tx, tw, bias, T, d, N, idx, gates, s);
+    default: return launch_router_tc_k<BN, STAGES, 8>(tx, tw, bias, T, d, N, idx, gates, s);
+  }
 }
 
 }  // namespace
@@ -477,17 +500,17 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(bucket_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BFMOE_MAX_EXPERTS * 4);
-    cudaFuncSetAttribute(bucket_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BFMOE_MAX_EXPERTS * 32);
+    cudaFuncSetAttribute(bucket_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         BFMOE_MAX_EXPERTS * 36 + 16);
     attr = true;
   }
   e = launch("bucket_count", s, [&] { bucket_count_kernel<<<nchunks, 1024, N * 4, s>>>(idx, R, N, cc); });
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket count");
   e = launch("bucket_scan", s, [&] { bucket_scan_kernel<<<(N + 31) / 32, 1024, 0, s>>>(cc, nchunks, N, totals); });
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scan");
-  e = launch("bucket_offsets", s, [&] { bucket_offsets_kernel<<<1, 1024, 0, s>>>(totals, N, counts, offsets); });
-  if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket offsets");
+  const size_t scatter_smem = ((N + 1) * 4 + 15) / 16 * 16 + static_cast<size_t>(N) * 32;
   e = launch("bucket_scatter", s, [&] {
-    bucket_scatter_kernel<<<nchunks, 1024, N * 32, s>>>(idx, R, N, cc, offsets, rows);
+    bucket_scatter_kernel<<<nchunks, 1024, scatter_smem, s>>>(idx, R, N, cc, totals, counts, offsets, rows);
   });
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scatter");
   return ok();
@@ -513,8 +536,8 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
   float2* tab_p = reinterpret_cast<float2*>(W + p.tab_phi);
   uint16_t* wbf = reinterpret_cast<uint16_t*>(W + p.w_bf16);
   void* xrot = W + p.xrot;
-  float* z = reinterpret_cast<float*>(W + p.z);
-  float* slot = reinterpret_cast<float*>(W + p.slot);
+  void* z = W + p.z;
+  void* slot = W + p.slot;
   const int L = ilog2(d);
   const long long R = static_cast<long long>(T) * k;
   const bool bf16 = x_dtype == BFMOE_BF16;
@@ -524,14 +547,11 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
   const bool fast = d >= 64;
   const long long nang = static_cast<long long>(N) * L * (d / 2);
   if (fast) {
-    const long long nq = nang / 2;
+    // one launch builds both tables; the phi table follows the theta table
     e = launch("rot_table", s, [&] {
-      rot_quads_kernel<<<grid_for(nq, 256, 8192), 256, 0, s>>>(layer->theta, N, d, L, reinterpret_cast<float4*>(tab_t));
+      rot_quads_kernel<<<2 * N * L, 256, 0, s>>>(layer->theta, layer->phi, N, d, L,
+                                                                  reinterpret_cast<float4*>(tab_t));
     });
-    if (e == cudaSuccess)
-      e = launch("rot_table", s, [&] {
-        rot_quads_kernel<<<grid_for(nq, 256, 8192), 256, 0, s>>>(layer->phi, N, d, L, reinterpret_cast<float4*>(tab_p));
-      });
   } else {
     e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->theta, nang, tab_t); });
     if (e == cudaSuccess)
@@ -554,9 +574,9 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
     if (!make_tmap_bf16(&ta, xrot, d, R, kGemmBM) || !make_tmap_bf16(&tb, wbf, d, d, BN))
       return fail(BFMOE_ECUDA, "forward: tensor map encoding failed");
     switch (BN) {
-      case 64: e = launch_gemm_tc<64, 8>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
-      case 128: e = launch_gemm_tc<128, 6>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
-      default: e = launch_gemm_tc<256, 4>(ta, tb, z, static_cast<int>(R), d, layer->alpha, s); break;
+      case 64: e = launch_gemm_tc<64, 8>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
+      case 128: e = launch_gemm_tc<128, 6>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
+      default: e = launch_gemm_tc<256, 4>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "forward: tensor-core GEMM");
   } else {
@@ -564,10 +584,11 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
     e = launch("ternary_gemm_simt", s, [&] {
       if (bf16)
         ternary_gemm_simt_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(xrot),
-                                                                  layer->w_packed, wpr, R, d, layer->alpha, z);
+                                                                  layer->w_packed, wpr, R, d, layer->alpha,
+                                                                  static_cast<float*>(z));
       else
         ternary_gemm_simt_kernel<float><<<g, 256, 0, s>>>(static_cast<const float*>(xrot), layer->w_packed, wpr, R,
-                                                          d, layer->alpha, z);
+                                                          d, layer->alpha, static_cast<float*>(z));
     });
     if (e != cudaSuccess) return cuda_fail(e, "forward: SIMT ternary product");
   }
@@ -578,11 +599,15 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
 
   const long long n4 = static_cast<long long>(T) * (d / 4);
   e = launch("combine", s, [&] {
-    if (bf16)
-      combine_kernel<__nv_bfloat16><<<grid_for(n4, 256, sm_count() * 16), 256, 0, s>>>(slot, T, k, d,
-                                                                                      static_cast<__nv_bfloat16*>(y));
+    const int g = grid_for(n4, 256, sm_count() * 16);
+    if (bf16 && fast)
+      combine_kernel<__nv_bfloat16, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(slot), T, k,
+                                                                     d, static_cast<__nv_bfloat16*>(y));
+    else if (bf16)
+      combine_kernel<float, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d,
+                                                             static_cast<__nv_bfloat16*>(y));
     else
-      combine_kernel<float><<<grid_for(n4, 256, sm_count() * 16), 256, 0, s>>>(slot, T, k, d, static_cast<float*>(y));
+      combine_kernel<float, float><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d, static_cast<float*>(y));
   });
   if (e != cudaSuccess) return cuda_fail(e, "forward: combine");
   return ok();

@@ -5,9 +5,9 @@
 // Rows are cut into chunks of kBucketChunk (one 1024-thread block each):
 //   count    per-chunk expert histogram
 //   scan     per expert, exclusive prefix over chunks (+ totals)
-//   offsets  exclusive prefix over experts (one block)
-//   scatter  position = offsets[e] + chunk prefix + earlier warps of the
-//            chunk + rank among equal experts inside the warp
+//   scatter  offsets = exclusive prefix over experts (each block); position =
+//            offsets[e] + chunk prefix + earlier warps of the chunk + rank
+//            among equal experts inside the warp
 #pragma once
 #include "common.cuh"
 
@@ -68,10 +68,9 @@ __global__ __launch_bounds__(1024) void bucket_scan_kernel(int32_t* __restrict__
     }
 }
 
-// One block of 1024 threads, N <= 4096 (4 experts per thread).
-__global__ __launch_bounds__(1024) void bucket_offsets_kernel(const int32_t* __restrict__ totals, int N,
-                                                              int32_t* __restrict__ counts,
-                                                              int32_t* __restrict__ offsets) {
+// Exclusive prefix sum of totals[0..N) into off[0..N] (shared memory), by a
+// block of 1024 threads, N <= 4096 (4 experts per thread).
+__device__ __forceinline__ void block_exclusive_scan(const int32_t* __restrict__ totals, int N, int* off) {
   __shared__ int warp_sum[32];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   int v[4];
@@ -84,44 +83,55 @@ __global__ __launch_bounds__(1024) void bucket_offsets_kernel(const int32_t* __r
   }
   int incl = local;
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(FULL_MASK, incl, off);
-    if (lane >= off) incl += o;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(FULL_MASK, incl, o);
+    if (lane >= o) incl += t;
   }
   if (lane == 31) warp_sum[w] = incl;
   __syncthreads();
   if (w == 0) {
-    int ws = warp_sum[lane];
+    const int ws = warp_sum[lane];
     int inc = ws;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(FULL_MASK, inc, off);
-      if (lane >= off) inc += o;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(FULL_MASK, inc, o);
+      if (lane >= o) inc += t;
     }
-    warp_sum[lane] = inc - ws;  // exclusive
+    warp_sum[lane] = inc - ws;
   }
   __syncthreads();
   int run = warp_sum[w] + incl - local;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int e = tid * 4 + q;
-    if (e < N) {
-      offsets[e] = run;
-      counts[e] = v[q];
-    }
+    if (e < N) off[e] = run;
     run += v[q];
   }
-  if (tid == 1023) offsets[N] = run;
+  if (tid == 1023) off[N] = run;
+  __syncthreads();
 }
 
+// Every block scans the per-expert totals itself (N <= 4096 ints), so the
+// offsets need no launch of their own; block 0 also writes counts and
+// offsets out.
 __global__ __launch_bounds__(1024) void bucket_scatter_kernel(const int32_t* __restrict__ idx, long long R, int N,
                                                               const int32_t* __restrict__ chunk_prefix,
-                                                              const int32_t* __restrict__ offsets,
+                                                              const int32_t* __restrict__ totals,
+                                                              int32_t* __restrict__ counts_out,
+                                                              int32_t* __restrict__ offsets_out,
                                                               int32_t* __restrict__ rows) {
-  extern __shared__ uint8_t wcnt[];  // [N][32]: rows of expert e in warp w
+  extern __shared__ uint8_t scatter_smem[];
+  int* off = reinterpret_cast<int*>(scatter_smem);                   // [N+1]
+  uint8_t* wcnt = scatter_smem + ((N + 1) * 4 + 15) / 16 * 16;       // [N][32]: rows of expert e in warp w
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   for (int q = tid; q < N * 8; q += blockDim.x) reinterpret_cast<uint32_t*>(wcnt)[q] = 0u;
-  __syncthreads();
+  block_exclusive_scan(totals, N, off);
+  if (blockIdx.x == 0) {
+    for (int e = tid; e <= N; e += blockDim.x) {
+      offsets_out[e] = off[e];
+      if (e < N) counts_out[e] = totals[e];
+    }
+  }
   const long long r = static_cast<long long>(blockIdx.x) * kBucketChunk + tid;
   int e = -1 - lane;
   bool valid = false;
@@ -142,7 +152,7 @@ __global__ __launch_bounds__(1024) void bucket_scatter_kernel(const int32_t* __r
   const int leader = __ffs(peers) - 1;
   before = __shfl_sync(FULL_MASK, before, leader);
   if (valid) {
-    const int pos = offsets[e] + chunk_prefix[static_cast<size_t>(blockIdx.x) * N + e] + before + rank;
+    const int pos = off[e] + chunk_prefix[static_cast<size_t>(blockIdx.x) * N + e] + before + rank;
     rows[pos] = static_cast<int32_t>(r);
   }
 }

@@ -10,10 +10,10 @@
 //                      swizzle) into a STAGES-deep shared-memory ring;
 //   warp 1 (one lane)  MMA issuer: tcgen05.mma M=128 N=BN K=16 into one of two
 //                      TMEM accumulators (2*BN columns);
-//   warps 2..5         epilogue: TMEM -> registers -> alpha * acc -> a per-warp
-//                      shared-memory transpose -> coalesced stores of Z; the
-//                      accumulator is released as soon as it is read, so the
-//                      next tile's MMAs overlap this tile's stores.
+//   warps 2..5         epilogue: TMEM -> registers -> alpha * acc rounded to
+//                      bf16 -> a per-warp shared-memory transpose -> coalesced
+//                      stores of Z; the accumulator is released as soon as it
+//                      is read, so the next tile's MMAs overlap these stores.
 #pragma once
 #include "common.cuh"
 
@@ -28,7 +28,7 @@ struct GemmTcCfg {
   static constexpr uint32_t A_BYTES = kGemmBM * kGemmBK * 2;
   static constexpr uint32_t B_BYTES = BN * kGemmBK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t EPI_BYTES = 4 * 32 * 32 * 4;  // 4 warps x 32x32 fp32
+  static constexpr uint32_t EPI_BYTES = 4 * 32 * 32 * 2;  // 4 warps x 32x32 bf16
   static constexpr uint32_t BAR_BYTES = (2 * STAGES + 4) * 8 + 8;
   static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -37,13 +37,13 @@ struct GemmTcCfg {
 template <int BN, int STAGES>
 __global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                                                                           const __grid_constant__ CUtensorMap tmB,
-                                                                          float* __restrict__ Z, int R, int d,
+                                                                          __nv_bfloat16* __restrict__ Z, int R, int d,
                                                                           float alpha) {
   using Cfg = GemmTcCfg<BN, STAGES>;
   static_assert(2 * BN == 64 || 2 * BN == 128 || 2 * BN == 256 || 2 * BN == 512, "TMEM columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* epi = reinterpret_cast<float*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint32_t* epi = reinterpret_cast<uint32_t*>(smem + STAGES * Cfg::STAGE_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES + Cfg::EPI_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;  // [2]
@@ -127,7 +127,7 @@ __global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const 
   } else {
     // epilogue warps 2..5: TMEM sub-partition (warp % 4) holds rows 32*(warp%4) ..
     const int sp = warp & 3;
-    float* buf_w = epi + (warp - 2) * 32 * 32;
+    uint32_t* buf_w = epi + (warp - 2) * 32 * 16;  // 32 rows x 16 bf16 pairs
     int i = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
       const int m0 = (t / n_tiles_n) * kGemmBM, n0 = (t % n_tiles_n) * BN;
@@ -147,20 +147,26 @@ __global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const 
           __syncwarp();
           if (lane == 0) mbar_arrive(tempty + buf);
         }
-        // lane = row: write 8 float4 (swizzled by row) ...
+        // lane = row: 16 bf16 pairs as 4 x 16 bytes, swizzled by row ...
+        uint32_t pk[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<float4*>(buf_w + lane * 32 + ((u ^ (lane & 7)) << 2)) =
-              make_float4(alpha * __uint_as_float(v[4 * u]), alpha * __uint_as_float(v[4 * u + 1]),
-                          alpha * __uint_as_float(v[4 * u + 2]), alpha * __uint_as_float(v[4 * u + 3]));
+        for (int j = 0; j < 16; ++j) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(alpha * __uint_as_float(v[2 * j]), alpha * __uint_as_float(v[2 * j + 1]));
+          pk[j] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        const int sw = (lane >> 1) & 3;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4*>(buf_w + lane * 16 + ((u ^ sw) << 2)) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         __syncwarp();
-        // ... then 4 rows x 128 bytes per store instruction
+        // ... then 8 rows x 64 bytes per store instruction
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int rr = q * 4 + (lane >> 3), u = lane & 7;
-          const float4 val = *reinterpret_cast<const float4*>(buf_w + rr * 32 + ((u ^ (rr & 7)) << 2));
+        for (int q = 0; q < 4; ++q) {
+          const int rr = q * 8 + (lane >> 2), u = lane & 3;
+          const uint4 val = *reinterpret_cast<const uint4*>(buf_w + rr * 16 + ((u ^ ((rr >> 1) & 3)) << 2));
           const int row = row0 + rr;
-          if (row < R) *reinterpret_cast<float4*>(Z + static_cast<size_t>(row) * d + n0 + c + 4 * u) = val;
+          if (row < R) *reinterpret_cast<uint4*>(Z + static_cast<size_t>(row) * d + n0 + c + 8 * u) = val;
         }
         __syncwarp();
       }

@@ -213,9 +213,9 @@ __global__ __launch_bounds__(256) void post_rotate_kernel(const float* __restric
   }
 }
 
-// y_t = sum_{j<k} slot[t*k + j] in slot order (float32), rounded once.
-template <typename Tout>
-__global__ __launch_bounds__(256) void combine_kernel(const float* __restrict__ slot, long long T, int k, int d,
+// y_t = sum_{j<k} slot[t*k + j] in slot order, in float32, rounded once.
+template <typename Ts, typename Tout>
+__global__ __launch_bounds__(256) void combine_kernel(const Ts* __restrict__ slot, long long T, int k, int d,
                                                       Tout* __restrict__ y) {
   const int d4 = d / 4;
   const long long n = T * d4;
@@ -223,21 +223,29 @@ __global__ __launch_bounds__(256) void combine_kernel(const float* __restrict__ 
        q += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long t = q / d4;
     const int c = static_cast<int>(q % d4) * 4;
-    const float* src = slot + static_cast<size_t>(t) * k * d + c;
-    float4 acc = __ldg(reinterpret_cast<const float4*>(src));
-    for (int j = 1; j < k; ++j) {
-      const float4 s = __ldg(reinterpret_cast<const float4*>(src + static_cast<size_t>(j) * d));
-      acc.x += s.x;
-      acc.y += s.y;
-      acc.z += s.z;
-      acc.w += s.w;
+    const Ts* src = slot + static_cast<size_t>(t) * k * d + c;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const Ts* sj = src + static_cast<size_t>(j) * d;
+      if constexpr (sizeof(Ts) == 4) {
+        const float4 s4 = __ldg(reinterpret_cast<const float4*>(sj));
+        acc[0] += s4.x;
+        acc[1] += s4.y;
+        acc[2] += s4.z;
+        acc[3] += s4.w;
+      } else {
+        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(sj));
+        const Ts* h = reinterpret_cast<const Ts*>(&raw);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[u] += to_f32(h[u]);
+      }
     }
     Tout* dst = y + static_cast<size_t>(t) * d + c;
     if constexpr (sizeof(Tout) == 4) {
-      *reinterpret_cast<float4*>(dst) = acc;
+      *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
     } else {
-      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
       uint2 raw;
       raw.x = *reinterpret_cast<uint32_t*>(&lo);
       raw.y = *reinterpret_cast<uint32_t*>(&hi);

@@ -11,11 +11,13 @@
 // loaded (cos, sin) to G rows of the same expert.
 //
 // Most stages process two rotations per packed float32 instruction
-// (__ffma2_rn / __fmul2_rn): the table stores, per stage, quads
-// (c_a, c_b, s_a, s_b) of the two rotations a lane pairs up.  Natural order
-// (a, b) = (2j, 2j+1) for layout-1 stages and stage 5; for layout-2 stages
-// s >= 6, quad qp*32 + l holds the rotations of lane l at registers q and q+1
-// (b = a + 32).
+// (__ffma2_rn / __fmul2_rn).  The cos/sin table stores, per stage, quads
+// (c_a, c_b, s_a, s_b) in the order the warp reads them: quad u*32 + l holds
+// the u-th pair of rotations that lane l applies, so each warp-wide table read
+// is 32 consecutive quads (no shared-memory bank conflicts).  A cross-lane
+// stage stores its slice for every lane (partner lanes hold the same
+// rotations), so it is twice the size of the others; layout-2 stage 5 keeps
+// the natural order (a, b) = (2j, 2j+1).
 #pragma once
 #include "common.cuh"
 #include "rotate.cuh"
@@ -30,7 +32,7 @@ struct Geo {
   static constexpr int P = e > 5 ? e : 5;
   static constexpr int D = 32 * E_;
   static constexpr int G = E_ <= 16 ? 4 : (E_ <= 32 ? 2 : 1);  // rows per warp
-  static constexpr int WARPS = 8;
+  static constexpr int WARPS = E_ <= 64 ? 8 : 4;
 };
 
 // Rotation index of element i in stage s (lower element of its pair).
@@ -38,32 +40,67 @@ __host__ __device__ __forceinline__ int rot_index(int i, int s) {
   return ((i >> (s + 1)) << s) + (i & ((1 << s) - 1));
 }
 
-// Quad table: [N][L][D/4] float4, layout described above.
-__global__ void rot_quads_kernel(const float* __restrict__ ang, int N, int d, int L, float4* __restrict__ quads) {
+// Quads of stage s in the table of one expert, for E elements per lane.
+__host__ __device__ constexpr int tab_stage_quads(int E, int s) {
+  int e = 0;
+  while ((1 << e) < E) ++e;
+  const int P = e > 5 ? e : 5;
+  if (s < P && s >= e) return 32 * (E / 2);            // cross-lane (layout 1)
+  if (s < P) return 32 * (E / 4 > 0 ? E / 4 : 1);      // in registers (layout 1)
+  return 8 * E;                                         // layout 2 (d/4)
+}
+__host__ __device__ constexpr int tab_stage_offset(int E, int s) {
+  int o = 0;
+  for (int i = 0; i < s; ++i) o += tab_stage_quads(E, i);
+  return o;
+}
+__host__ __device__ constexpr int tab_quads(int E) {
+  int e = 0;
+  while ((1 << e) < E) ++e;
+  return tab_stage_offset(E, e + 5);
+}
+
+// Quad tables: [2][N][tab_quads(E)] float4 (theta then phi).  One block per
+// (table, expert, stage), one thread per quad.
+__global__ __launch_bounds__(256) void rot_quads_kernel(const float* __restrict__ theta,
+                                                        const float* __restrict__ phi, int N, int d, int L,
+                                                        float4* __restrict__ quads) {
+  const int E = d / 32;
   const int e = L - 5;
   const int P = e > 5 ? e : 5;
-  const long long per_stage = d / 4;
-  const long long n = static_cast<long long>(N) * L * per_stage;
-  for (long long q = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; q < n;
-       q += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int Q = static_cast<int>(q % per_stage);
-    const int s = static_cast<int>((q / per_stage) % L);
-    const long long ex = q / (per_stage * L);
+  const int s = blockIdx.x % L;
+  const int ex = (blockIdx.x / L) % N;
+  const int which = blockIdx.x / (L * N);
+  const float* base = (which ? phi : theta) + (static_cast<size_t>(ex) * L + s) * (d / 2);
+  float4* out = quads + (static_cast<size_t>(which) * N + ex) * tab_quads(E) + tab_stage_offset(E, s);
+  const int nq = tab_stage_quads(E, s);
+  for (int Q = threadIdx.x; Q < nq; Q += blockDim.x) {
+    const int lane = Q & 31, u = Q >> 5;
     int a, b;
-    if (s < P || s == 5) {
+    if (s < P && s >= e) {  // cross-lane: rotations base + 2u, base + 2u + 1
+      const int m = 1 << (s - e);
+      const int i_lo = (lane & ~m) * E;
+      a = rot_index(i_lo, s) + 2 * u;
+      b = a + 1;
+    } else if (s == 0) {  // layout 1, pairs (q, q+1): rotations l*E/2 + 2u, +1
+      a = lane * (E / 2) + 2 * u;
+      b = E >= 4 ? a + 1 : a;
+    } else if (s < P) {  // layout 1 in registers: the u-th even q with bit s clear
+      const int q = ((u >> (s - 1)) << (s + 1)) | ((u & ((1 << (s - 1)) - 1)) << 1);
+      a = lane * (E / 2) + ((q >> (s + 1)) << s) + (q & ((1 << s) - 1));
+      b = a + 1;
+    } else if (s == 5) {  // layout 2, stage 5: natural order
       a = 2 * Q;
       b = a + 1;
-    } else {
-      const int lane = Q & 31, qp = Q >> 5;
-      const int qq = ((qp >> (s - 6)) << (s - 4)) | ((qp & ((1 << (s - 6)) - 1)) << 1);
+    } else {  // layout 2, s >= 6: lane l's registers q and q+1 (b = a + 32)
+      const int qq = ((u >> (s - 6)) << (s - 4)) | ((u & ((1 << (s - 6)) - 1)) << 1);
       a = ((qq >> (s - 4)) << s) | ((qq & ((1 << (s - 5)) - 1)) << 5) | lane;
       b = a + 32;
     }
-    const float* base = ang + (ex * L + s) * static_cast<long long>(d / 2);
     float sa, ca, sb, cb;
     sincosf(base[a], &sa, &ca);
     sincosf(base[b], &sb, &cb);
-    quads[q] = make_float4(ca, cb, sa, sb);
+    out[Q] = make_float4(ca, cb, sa, sb);
   }
 }
 
@@ -76,10 +113,10 @@ template <int E, int G, bool TR>
 __device__ __forceinline__ void l1_stage0(float (&v)[G][E], const float4* __restrict__ tq, int lane) {
 #pragma unroll
   for (int q = 0; q < E; q += 2) {
-    const int r = lane * (E / 2) + (q >> 1);
-    const float4 qd = __ldg(tq + (r >> 1));
-    const float c = (r & 1) ? qd.y : qd.x;
-    const float s = (r & 1) ? qd.w : qd.z;
+    const float4 qd = tq[(q >> 2) * 32 + lane];
+    const bool hi = (q >> 1) & 1;
+    const float c = hi ? qd.y : qd.x;
+    const float s = hi ? qd.w : qd.z;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const float a = v[g][q], b = v[g][q + 1];
@@ -98,11 +135,12 @@ __device__ __forceinline__ void l1_stage0(float (&v)[G][E], const float4* __rest
 template <int E, int G, int S, bool TR>
 __device__ __forceinline__ void l1_stage_reg(float (&v)[G][E], const float4* __restrict__ tq, int lane) {
   constexpr int h = 1 << S;
+  int u = 0;
 #pragma unroll
   for (int q = 0; q < E; q += 2) {
     if (q & h) continue;
-    const int r = lane * (E / 2) + ((q >> (S + 1)) << S) + (q & (h - 1));
-    const float4 qd = __ldg(tq + (r >> 1));
+    const float4 qd = tq[u * 32 + lane];
+    ++u;
     const float2 c = make_float2(qd.x, qd.y);
     const float2 s = make_float2(qd.z, qd.w);
     const float2 ns = f2neg(s);
@@ -132,13 +170,11 @@ __device__ __forceinline__ void l1_stage_cross(float (&v)[G][E], const float4* _
   constexpr int e = Log2<E>::value;
   constexpr int m = 1 << (s - e);
   const bool upper = (lane & m) != 0;
-  const int i_lo = (lane & ~m) * E;
-  const int base = rot_index(i_lo, s);
   // own' = c*own + sg*partner with sg = (upper ? s : -s) forward, (upper ? -s : s) transposed
   const bool neg = TR ? upper : !upper;
 #pragma unroll
   for (int q = 0; q < E; q += 2) {
-    const float4 qd = __ldg(tq + ((base + q) >> 1));
+    const float4 qd = tq[(q >> 1) * 32 + lane];
     const float2 c = make_float2(qd.x, qd.y);
     const float2 sg = neg ? make_float2(-qd.z, -qd.w) : make_float2(qd.z, qd.w);
 #pragma unroll
@@ -160,7 +196,7 @@ __device__ __forceinline__ void l2_stage5(float (&v)[G][E], const float4* __rest
 #pragma unroll
   for (int q = 0; q < E; q += 2) {
     const int r = 32 * (q >> 1) + lane;
-    const float4 qd = __ldg(tq + (r >> 1));
+    const float4 qd = tq[r >> 1];
     const float c = (r & 1) ? qd.y : qd.x;
     const float s = (r & 1) ? qd.w : qd.z;
 #pragma unroll
@@ -185,7 +221,7 @@ __device__ __forceinline__ void l2_stage_reg(float (&v)[G][E], const float4* __r
 #pragma unroll
   for (int q = 0; q < E; q += 2) {
     if (q & h) continue;
-    const float4 qd = __ldg(tq + qp * 32 + lane);
+    const float4 qd = tq[qp * 32 + lane];
     ++qp;
     const float2 c = make_float2(qd.x, qd.y);
     const float2 sn = make_float2(qd.z, qd.w);
@@ -214,7 +250,7 @@ __device__ __forceinline__ void l2_stage_reg(float (&v)[G][E], const float4* __r
 
 template <class Gm, int G, int s, bool TR>
 __device__ __forceinline__ void l1_stage(float (&v)[G][Gm::E], const float4* __restrict__ tq, int lane) {
-  const float4* t = tq + static_cast<size_t>(s) * (Gm::D / 4);
+  const float4* t = tq + tab_stage_offset(Gm::E, s);
   if constexpr (s == 0) {
     l1_stage0<Gm::E, G, TR>(v, t, lane);
   } else if constexpr (s < Gm::e) {
@@ -225,7 +261,7 @@ __device__ __forceinline__ void l1_stage(float (&v)[G][Gm::E], const float4* __r
 }
 template <class Gm, int G, int s, bool TR>
 __device__ __forceinline__ void l2_stage(float (&v)[G][Gm::E], const float4* __restrict__ tq, int lane) {
-  const float4* t = tq + static_cast<size_t>(s) * (Gm::D / 4);
+  const float4* t = tq + tab_stage_offset(Gm::E, s);
   if constexpr (s == 5) {
     l2_stage5<Gm::E, G, TR>(v, t, lane);
   } else {
@@ -308,21 +344,78 @@ __device__ __forceinline__ void to_layout1(float (&r)[E], float* buf, int lane) 
   __syncwarp();
 }
 
-// ---- kernels ------------------------------------------------------------------------
+// ---- kernels: rows and cos/sin tables staged in shared memory ------------------
+//
+// A CTA takes ROWS = WARPS * G consecutive bucket positions.  It first copies
+// the gathered input rows and the cos/sin tables of the first and last expert
+// of its range (bucket order sorts rows by expert) into shared memory with
+// cp.async, so the global-load latency of one CTA overlaps the arithmetic of
+// the others on the SM; warp w then rotates rows [w*G, w*G + G).
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// 16-byte chunk c of a staged float32 row sits at chunk c ^ ((c >> 3) & 7):
+// layout-1 float4 reads of 8 lanes then hit 8 different bank groups.
+__device__ __forceinline__ int chunk_swz(int c) { return c ^ ((c >> 3) & 7); }
+
+template <int E, typename Tin>
+struct StagedCfg {
+  using Gm = Geo<E>;
+  static constexpr int G = Gm::G;
+  static constexpr int ROWS = Gm::WARPS * G;
+  static constexpr int THREADS = Gm::WARPS * 32;
+  static constexpr size_t TAB_QUADS = tab_quads(E);
+  // expert tables kept in shared memory (18 KB each at d=512) while two CTAs
+  // still fit on an SM; larger widths read them through L1
+  static constexpr int NTAB = Gm::D <= 512 ? (sizeof(Tin) == 2 ? 2 : 1) : (Gm::D <= 1024 && sizeof(Tin) == 2 ? 1 : 0);
+  static constexpr size_t SMEM = ROWS * Gm::D * sizeof(Tin) + NTAB * TAB_QUADS * 16 + Gm::WARPS * Gm::D * 4 +
+                                 ROWS * 12 + 64;
+};
+
+struct RowMeta {
+  int row;    // routed row r = t*k + j (or -1)
+  int ex;     // expert (or -1)
+  float gate;
+};
+
+// Stage the tables of the first and last expert of the CTA's range; returns
+// where each row's table lives (shared memory when staged, else global).
+template <class C>
+__device__ __forceinline__ const float4* table_for(int e, int ea, int eb, const float4* smem_tab,
+                                                   const float4* __restrict__ quads) {
+  if (C::NTAB >= 1 && e == ea) return smem_tab;
+  if (C::NTAB >= 2 && e == eb) return smem_tab + C::TAB_QUADS;
+  return quads + static_cast<size_t>(e) * C::TAB_QUADS;
+}
+
+template <class C>
+__device__ __forceinline__ void stage_tables(int ea, int eb, float4* smem_tab, const float4* __restrict__ quads) {
+  if constexpr (C::NTAB >= 1) {
+    if (ea >= 0)
+      for (size_t i = threadIdx.x; i < C::TAB_QUADS; i += blockDim.x)
+        cp_async16(smem_tab + i, quads + static_cast<size_t>(ea) * C::TAB_QUADS + i);
+  }
+  if constexpr (C::NTAB >= 2) {
+    if (eb >= 0 && eb != ea)
+      for (size_t i = threadIdx.x; i < C::TAB_QUADS; i += blockDim.x)
+        cp_async16(smem_tab + C::TAB_QUADS + i, quads + static_cast<size_t>(eb) * C::TAB_QUADS + i);
+  }
+}
 
 template <class Gm, int G, typename Tin, typename Tout>
-__device__ __forceinline__ void pre_rotate_rows(const Tin* __restrict__ x, const int (&tok)[G],
-                                                const float4* __restrict__ tq, Tout* __restrict__ dst0,
-                                                float* buf, int lane) {
+__device__ __forceinline__ void pre_rotate_rows_smem(const Tin* xs0, const float4* tq, Tout* __restrict__ dst0,
+                                                     float* buf, int lane) {
   constexpr int E = Gm::E;
   float v[G][E];
-  // load in layout 2: element q*32 + lane (each warp load covers 32 consecutive elements)
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const Tin* src = x + static_cast<size_t>(tok[g]) * Gm::D + lane;
+  for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int q = 0; q < E; ++q) v[g][q] = to_f32(src[q * 32]);
-  }
+    for (int q = 0; q < E; ++q) v[g][q] = to_f32(xs0[g * Gm::D + q * 32 + lane]);  // layout 2
   l2_tr<Gm, G, Gm::L - 1>(v, tq, lane);
 #pragma unroll
   for (int g = 0; g < G; ++g) to_layout1<E>(v[g], buf, lane);
@@ -332,142 +425,192 @@ __device__ __forceinline__ void pre_rotate_rows(const Tin* __restrict__ x, const
 }
 
 // xrot[p] = B(theta_e)^T x_t for bucket positions p (row r = rows[p],
-// t = r / k, e = idx[r]); each warp takes G consecutive positions.
+// t = r / k, e = idx[r]).
 template <int E, typename Tin, typename Tout>
-__global__ __launch_bounds__(256) void pre_rotate_fast_kernel(const Tin* __restrict__ x,
+__global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS) void pre_rotate_fast_kernel(const Tin* __restrict__ x,
                                                               const int32_t* __restrict__ idx,
                                                               const int32_t* __restrict__ rows,
                                                               const float4* __restrict__ quads, long long R, int k,
                                                               int N, Tout* __restrict__ xrot) {
-  using Gm = Geo<E>;
-  constexpr int G = Gm::G;
-  extern __shared__ __align__(16) float sbuf[];
+  using C = StagedCfg<E, Tin>;
+  using Gm = typename C::Gm;
+  constexpr int G = C::G, ROWS = C::ROWS, D = Gm::D;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Tin* xs = reinterpret_cast<Tin*>(smem_raw);
+  float4* tab = reinterpret_cast<float4*>(smem_raw + ROWS * D * sizeof(Tin));
+  float* tbuf = reinterpret_cast<float*>(smem_raw + ROWS * D * sizeof(Tin) + C::NTAB * C::TAB_QUADS * 16);
+  RowMeta* meta = reinterpret_cast<RowMeta*>(tbuf + Gm::WARPS * D);
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  float* buf = sbuf + w * Gm::D;
-  const long long p0 = (static_cast<long long>(blockIdx.x) * Gm::WARPS + w) * G;
-  if (p0 >= R) return;
-  const size_t stage_quads = static_cast<size_t>(Gm::L) * (Gm::D / 4);
-  int tok[G], ex[G];
-  bool ok = true;
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const long long p = p0 + g;
-    tok[g] = 0;
-    ex[g] = -1;
+  const long long p0 = static_cast<long long>(blockIdx.x) * ROWS;
+
+  if (threadIdx.x < ROWS) {
+    const long long p = p0 + threadIdx.x;
+    RowMeta m{-1, -1, 0.f};
     if (p < R) {
       const int r = rows[p];
       if (r >= 0 && r < R) {
         const int e = idx[r];
-        if (e >= 0 && e < N) {
-          ex[g] = e;
-          tok[g] = r / k;
-        }
+        if (e >= 0 && e < N) m = RowMeta{r, e, 0.f};
       }
-      if (ex[g] < 0) ok = false;
+      if (m.ex < 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
     }
+    meta[threadIdx.x] = m;
   }
-  bool same = ok;
+  __syncthreads();
+  // first and last expert of the range (rows are sorted by expert)
+  static_assert(ROWS <= 32, "one warp ballot covers the range");
+  const int my_ex = lane < ROWS ? meta[lane].ex : -1;
+  const unsigned vm = __ballot_sync(FULL_MASK, my_ex >= 0);
+  const int ea = vm ? __shfl_sync(FULL_MASK, my_ex, __ffs(vm) - 1) : -1;
+  const int eb = vm ? __shfl_sync(FULL_MASK, my_ex, 31 - __clz(vm)) : -1;
+  // gathered input rows (invalid rows read token 0; their output is zeroed)
+  constexpr int CH = D * sizeof(Tin) / 16;
+  for (int i = threadIdx.x; i < ROWS * CH; i += blockDim.x) {
+    const int rr = i / CH, c = i % CH;
+    const int rid = meta[rr].row;
+    const int t = rid >= 0 ? rid / k : 0;
+    cp_async16(reinterpret_cast<uint8_t*>(xs) + static_cast<size_t>(rr) * D * sizeof(Tin) + c * 16,
+               reinterpret_cast<const uint8_t*>(x + static_cast<size_t>(t) * D) + c * 16);
+  }
+  stage_tables<C>(ea, eb, tab, quads);
+  cp_async_wait_all();
+  __syncthreads();
+
+  float* buf = tbuf + w * D;
+  const int r0 = w * G;
+  if (p0 + r0 >= R) return;
+  bool same = p0 + r0 + G <= R;
 #pragma unroll
-  for (int g = 1; g < G; ++g)
-    if (p0 + g < R && ex[g] != ex[0]) same = false;
-  if (same && p0 + G <= R) {
-    pre_rotate_rows<Gm, G, Tin, Tout>(x, tok, quads + ex[0] * stage_quads, xrot + p0 * Gm::D, buf, lane);
+  for (int g = 0; g < G; ++g)
+    if (meta[r0 + g].ex < 0 || meta[r0 + g].ex != meta[r0].ex) same = false;
+  if (same) {
+    pre_rotate_rows_smem<Gm, G, Tin, Tout>(xs + r0 * D, table_for<C>(meta[r0].ex, ea, eb, tab, quads),
+                                           xrot + (p0 + r0) * D, buf, lane);
     return;
   }
 #pragma unroll 1
   for (int g = 0; g < G; ++g) {
-    const long long p = p0 + g;
+    const long long p = p0 + r0 + g;
     if (p >= R) break;
-    if (ex[g] < 0) {
-      if (lane == 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
+    const int e = meta[r0 + g].ex;
+    if (e < 0) {
       float z[E];
 #pragma unroll
       for (int q = 0; q < E; ++q) z[q] = 0.f;
-      store_row<E, Tout>(xrot + p * Gm::D + lane * E, z, true);
+      store_row<E, Tout>(xrot + p * D + lane * E, z, true);
       continue;
     }
-    const int t1[1] = {tok[g]};
-    pre_rotate_rows<Gm, 1, Tin, Tout>(x, t1, quads + ex[g] * stage_quads, xrot + p * Gm::D, buf, lane);
+    pre_rotate_rows_smem<Gm, 1, Tin, Tout>(xs + (r0 + g) * D, table_for<C>(e, ea, eb, tab, quads), xrot + p * D,
+                                           buf, lane);
   }
 }
 
-template <class Gm, int G>
-__device__ __forceinline__ void post_rotate_rows(const float* __restrict__ z0, const float4* __restrict__ tq,
-                                                 const int (&row)[G], const float (&gate)[G],
-                                                 float* __restrict__ slot, float* buf, int lane) {
+template <class Gm, int G, typename Tz, typename Ts>
+__device__ __forceinline__ void post_rotate_rows_smem(const Tz* zs0, const float4* tq, const RowMeta* m,
+                                                      Ts* __restrict__ slot, float* buf, int lane) {
   constexpr int E = Gm::E;
+  constexpr int PER = 16 / sizeof(Tz);  // elements per 16-byte chunk
   float v[G][E];
 #pragma unroll
-  for (int g = 0; g < G; ++g) load_row<E, float>(z0 + static_cast<size_t>(g) * Gm::D + lane * E, v[g], true);
+  for (int g = 0; g < G; ++g) {
+    const uint8_t* zr = reinterpret_cast<const uint8_t*>(zs0 + g * Gm::D);
+    if constexpr (E % PER == 0) {
+#pragma unroll
+      for (int u = 0; u < E / PER; ++u) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(zr + 16 * chunk_swz(lane * (E / PER) + u));
+        const Tz* t = reinterpret_cast<const Tz*>(&raw);
+#pragma unroll
+        for (int j = 0; j < PER; ++j) v[g][u * PER + j] = to_f32(t[j]);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < E; ++q) {
+        const int i = lane * E + q;
+        v[g][q] = to_f32(*reinterpret_cast<const Tz*>(zr + 16 * chunk_swz(i / PER) + (i % PER) * sizeof(Tz)));
+      }
+    }
+  }
   l1_fwd<Gm, G, 0>(v, tq, lane);
 #pragma unroll
   for (int g = 0; g < G; ++g) to_layout2<E>(v[g], buf, lane);
   l2_fwd<Gm, G, Gm::P>(v, tq, lane);
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    float* dst = slot + static_cast<size_t>(row[g]) * Gm::D + lane;
+    Ts* dst = slot + static_cast<size_t>(m[g].row) * Gm::D + lane;
+    const float gt = m[g].gate;
 #pragma unroll
-    for (int q = 0; q < E; ++q) dst[q * 32] = gate[g] * v[g][q];
+    for (int q = 0; q < E; ++q) dst[q * 32] = from_f32<Ts>(gt * v[g][q]);
   }
 }
 
-// slot[r] = g_r * B(phi_e) z_p for bucket positions p; G positions per warp.
-template <int E>
-__global__ __launch_bounds__(256) void post_rotate_fast_kernel(const float* __restrict__ z,
-                                                               const int32_t* __restrict__ idx,
-                                                               const float* __restrict__ gates,
-                                                               const int32_t* __restrict__ rows,
-                                                               const float4* __restrict__ quads, long long R, int N,
-                                                               float* __restrict__ slot) {
-  using Gm = Geo<E>;
-  constexpr int G = Gm::G;
-  extern __shared__ __align__(16) float sbuf[];
+// slot[r] = g_r * B(phi_e) z_p for bucket positions p (z already scaled by
+// alpha), r = rows[p], e = idx[r].
+template <int E, typename Tz, typename Ts>
+__global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS) void post_rotate_fast_kernel(
+    const Tz* __restrict__ z, const int32_t* __restrict__ idx, const float* __restrict__ gates,
+    const int32_t* __restrict__ rows, const float4* __restrict__ quads, long long R, int N, Ts* __restrict__ slot) {
+  using C = StagedCfg<E, Tz>;
+  using Gm = typename C::Gm;
+  constexpr int G = C::G, ROWS = C::ROWS, D = Gm::D;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Tz* zs = reinterpret_cast<Tz*>(smem_raw);
+  float4* tab = reinterpret_cast<float4*>(smem_raw + ROWS * D * sizeof(Tz));
+  float* tbuf = reinterpret_cast<float*>(smem_raw + ROWS * D * sizeof(Tz) + C::NTAB * C::TAB_QUADS * 16);
+  RowMeta* meta = reinterpret_cast<RowMeta*>(tbuf + Gm::WARPS * D);
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  float* buf = sbuf + w * Gm::D;
-  const long long p0 = (static_cast<long long>(blockIdx.x) * Gm::WARPS + w) * G;
-  if (p0 >= R) return;
-  const size_t stage_quads = static_cast<size_t>(Gm::L) * (Gm::D / 4);
-  int row[G], ex[G];
-  float gate[G];
-  bool ok = true;
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const long long p = p0 + g;
-    row[g] = 0;
-    ex[g] = -1;
-    gate[g] = 0.f;
+  const long long p0 = static_cast<long long>(blockIdx.x) * ROWS;
+
+  if (threadIdx.x < ROWS) {
+    const long long p = p0 + threadIdx.x;
+    RowMeta m{-1, -1, 0.f};
     if (p < R) {
       const int r = rows[p];
       if (r >= 0 && r < R) {
         const int e = idx[r];
-        if (e >= 0 && e < N) {
-          ex[g] = e;
-          row[g] = r;
-          gate[g] = gates[r];
-        }
+        if (e >= 0 && e < N) m = RowMeta{r, e, gates[r]};
       }
-      if (ex[g] < 0) ok = false;
+      if (m.ex < 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
     }
+    meta[threadIdx.x] = m;
   }
-  bool same = ok;
+  __syncthreads();
+  // first and last expert of the range (rows are sorted by expert)
+  static_assert(ROWS <= 32, "one warp ballot covers the range");
+  const int my_ex = lane < ROWS ? meta[lane].ex : -1;
+  const unsigned vm = __ballot_sync(FULL_MASK, my_ex >= 0);
+  const int ea = vm ? __shfl_sync(FULL_MASK, my_ex, __ffs(vm) - 1) : -1;
+  const int eb = vm ? __shfl_sync(FULL_MASK, my_ex, 31 - __clz(vm)) : -1;
+  constexpr int CH = D * sizeof(Tz) / 16;  // 16-byte chunks per row
+  for (int i = threadIdx.x; i < ROWS * CH; i += blockDim.x) {
+    const int rr = i / CH, c = i % CH;
+    const long long p = p0 + rr < R ? p0 + rr : R - 1;
+    cp_async16(reinterpret_cast<uint8_t*>(zs) + static_cast<size_t>(rr) * D * sizeof(Tz) + 16 * chunk_swz(c),
+               reinterpret_cast<const uint8_t*>(z + p * D) + 16 * c);
+  }
+  stage_tables<C>(ea, eb, tab, quads);
+  cp_async_wait_all();
+  __syncthreads();
+
+  float* buf = tbuf + w * D;
+  const int r0 = w * G;
+  if (p0 + r0 >= R) return;
+  bool same = p0 + r0 + G <= R;
 #pragma unroll
-  for (int g = 1; g < G; ++g)
-    if (p0 + g < R && ex[g] != ex[0]) same = false;
-  if (same && p0 + G <= R) {
-    post_rotate_rows<Gm, G>(z + p0 * Gm::D, quads + ex[0] * stage_quads, row, gate, slot, buf, lane);
+  for (int g = 0; g < G; ++g)
+    if (meta[r0 + g].ex < 0 || meta[r0 + g].ex != meta[r0].ex) same = false;
+  if (same) {
+    post_rotate_rows_smem<Gm, G, Tz, Ts>(zs + r0 * D, table_for<C>(meta[r0].ex, ea, eb, tab, quads), meta + r0,
+                                         slot, buf, lane);
     return;
   }
 #pragma unroll 1
   for (int g = 0; g < G; ++g) {
-    const long long p = p0 + g;
+    const long long p = p0 + r0 + g;
     if (p >= R) break;
-    if (ex[g] < 0) {
-      if (lane == 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
-      continue;
-    }
-    const int r1[1] = {row[g]};
-    const float g1[1] = {gate[g]};
-    post_rotate_rows<Gm, 1>(z + p * Gm::D, quads + ex[g] * stage_quads, r1, g1, slot, buf, lane);
+    const int e = meta[r0 + g].ex;
+    if (e < 0) continue;
+    post_rotate_rows_smem<Gm, 1, Tz, Ts>(zs + (r0 + g) * D, table_for<C>(e, ea, eb, tab, quads), meta + r0 + g,
+                                         slot, buf, lane);
   }
 }
 

@@ -49,11 +49,41 @@ struct RouterTcCfg {
 
 constexpr int kRouterThreads = 192;
 
-template <int BN, int STAGES>
+// Running top-K of one row in registers (K compile-time): larger logit first,
+// lower expert index first on equal logits.
+template <int K>
+struct TopK {
+  float v[K];
+  int id[K];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      v[j] = -INFINITY;
+      id[j] = 0x7fffffff;
+    }
+  }
+  __device__ __forceinline__ void push(float l, int e) {
+    if (!ranks_before(l, e, v[K - 1], id[K - 1])) return;
+    float cv = l;
+    int ci = e;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      const bool sw = ranks_before(cv, ci, v[j], id[j]);
+      const float tv = v[j];
+      const int ti = id[j];
+      v[j] = sw ? cv : tv;
+      id[j] = sw ? ci : ti;
+      cv = sw ? tv : cv;
+      ci = sw ? ti : ci;
+    }
+  }
+};
+
+template <int BN, int STAGES, int K>
 __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                                                            const __grid_constant__ CUtensorMap tmW,
                                                            const float* __restrict__ bias, int T, int d, int N,
-                                                           int k, int32_t* __restrict__ idx,
+                                                           int32_t* __restrict__ idx,
                                                            float* __restrict__ gates) {
   using Cfg = RouterTcCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -149,15 +179,8 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
   // Epilogue (warps 2..5): one token row per thread.
   const int sp = warp & 3;
   const int row = m0 + sp * 32 + lane;
-  float v[BFMOE_MAX_K];
-  int id[BFMOE_MAX_K];
-#pragma unroll
-  for (int j = 0; j < BFMOE_MAX_K; ++j) {
-    v[j] = -INFINITY;
-    id[j] = 0x7fffffff;
-  }
-  float th_v = -INFINITY;
-  int th_i = 0x7fffffff;
+  TopK<K> top;
+  top.init();
   bool ok = true;
   for (int c = 0; c < nchunks; ++c) {
     const int buf = c & 1;
@@ -169,33 +192,18 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
     const uint32_t base = tmem + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(buf * BN);
 #pragma unroll 1
     for (int col = 0; col < BN; col += 32) {
+      const int e0 = c * BN + col;
+      float b[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) b[q] = (e0 + q < N) ? (bias ? __ldg(bias + e0 + q) : 0.f) : -INFINITY;
       uint32_t r[32];
       tmem_ld_32x32b_x32(base + static_cast<uint32_t>(col), r);
       tmem_wait_ld();
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
-        const int e = c * BN + col + q;
-        if (e >= N) break;
-        float l = __uint_as_float(r[q]) + (bias ? __ldg(bias + e) : 0.f);
+        float l = __uint_as_float(r[q]) + b[q];
         if (isnan(l)) l = -INFINITY;
-        if (!ranks_before(l, e, th_v, th_i)) continue;
-        float cv = l;
-        int ci = e;
-#pragma unroll
-        for (int j = 0; j < BFMOE_MAX_K; ++j) {
-          if (j < k && ranks_before(cv, ci, v[j], id[j])) {
-            const float tv = v[j];
-            const int ti = id[j];
-            v[j] = cv;
-            id[j] = ci;
-            cv = tv;
-            ci = ti;
-          }
-          if (j == k - 1) {
-            th_v = v[j];
-            th_i = id[j];
-          }
-        }
+        top.push(l, e0 + q < N ? e0 + q : 0x7fffffff);
       }
     }
     tc_fence_before();
@@ -203,20 +211,18 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
     if (lane == 0) mbar_arrive(acc_empty + buf);
   }
   if (ok && row < T) {
-    float z[BFMOE_MAX_K];
+    float z[K];
     float sum = 0.f;
-    const bool finite_top = v[0] > -INFINITY;
+    const bool finite_top = top.v[0] > -INFINITY;
 #pragma unroll
-    for (int j = 0; j < BFMOE_MAX_K; ++j) {
-      if (j >= k) break;
-      z[j] = finite_top ? expf(v[j] - v[0]) : 1.f;
+    for (int j = 0; j < K; ++j) {
+      z[j] = finite_top ? expf(top.v[j] - top.v[0]) : 1.f;
       sum += z[j];
     }
 #pragma unroll
-    for (int j = 0; j < BFMOE_MAX_K; ++j) {
-      if (j >= k) break;
-      idx[static_cast<size_t>(row) * k + j] = id[j];
-      gates[static_cast<size_t>(row) * k + j] = z[j] / sum;
+    for (int j = 0; j < K; ++j) {
+      idx[static_cast<size_t>(row) * K + j] = top.id[j];
+      gates[static_cast<size_t>(row) * K + j] = z[j] / sum;
     }
   }
   tc_fence_before();
