@@ -133,10 +133,13 @@ class ClockSampler:
 # Algorithmic cost of each kernel, per launch (the roofline numerators)
 # ---------------------------------------------------------------------------
 def kernel_costs(wl, tables_bytes):
+    """Algorithmic work per launch of each kernel: (bound, amount, unit).
+    ``tables_bytes`` is one cos/sin table set (N L d/2 rotations x 8 bytes)."""
     d, N, k, T = wl.d, wl.n_experts, wl.k, wl.tokens
     R = T * k
     L = wl.stages
     xb = 2 if wl.dtype == "bf16" else 4
+    ib = 2 if (wl.dtype == "bf16" and d >= 64) else 4  # Z and slot element size
     return {
         # GEMM: 2 R d^2 flops on the tensor cores
         "ternary_gemm_tc": ("tensor", 2.0 * R * d * d, "TFLOP/s"),
@@ -149,10 +152,11 @@ def kernel_costs(wl, tables_bytes):
         "router_split": ("hbm", N * d * 4 + 3 * N * d * 2, "GB/s"),
         # pre-rotation: x rows gathered (R rows) + X_rot written + the theta table
         "pre_rotate": ("hbm", R * d * xb + R * d * xb + tables_bytes, "GB/s"),
-        # post-rotation: Z read (fp32) + slots written (fp32) + the phi table
-        "post_rotate": ("hbm", R * d * 4 + R * d * 4 + tables_bytes, "GB/s"),
-        "combine": ("hbm", R * d * 4 + T * d * xb, "GB/s"),
-        "rot_table": ("hbm", N * L * (d // 2) * 4 + tables_bytes, "GB/s"),
+        # post-rotation: Z read + gated slots written + the phi table
+        "post_rotate": ("hbm", R * d * ib + R * d * ib + tables_bytes, "GB/s"),
+        "combine": ("hbm", R * d * ib + T * d * xb, "GB/s"),
+        "rot_table": ("hbm", 2 * N * L * (d // 2) * 4 + 2 * tables_bytes, "GB/s"),
+        "expand_base_bf16": ("hbm", d * d // 4 + 2 * d * d, "GB/s"),
         "router_topk": ("hbm", T * N * 4 + T * k * 8, "GB/s"),
     }
 
@@ -332,8 +336,7 @@ def run_ours(args, wl):
         T = wl.tokens
         value = T * world * args.steps / (total_ms / 1e3)
         L = wl.stages
-        tables = 2 * wl.n_experts * L * (wl.d // 2) * 8
-        costs = kernel_costs(wl, tables // 2)
+        costs = kernel_costs(wl, wl.n_experts * L * (wl.d // 2) * 8)
         kernels = {}
         for name, (n, ms) in kt.items():
             entry = {"launches": n, "total_ms": ms, "share": ms / max(1e-9, sum(v[1] for v in kt.values())),

@@ -316,8 +316,9 @@ struct PostRotateFast {
     }
     const float4* q = reinterpret_cast<const float4*>(a.cs);
     return launch("post_rotate", a.s, [&] {
-      post_rotate_fast_kernel<E, T, T><<<static_cast<int>((a.R + C::ROWS - 1) / C::ROWS), C::THREADS, C::SMEM, a.s>>>(
-          static_cast<const T*>(a.z), a.idx, a.gates, a.rows, q, a.R, a.N, static_cast<T*>(a.out));
+      post_rotate_fast_kernel<E, T, T><<<static_cast<int>((a.R + C::ROWS - 1) / C::ROWS), C::THREADS, C::SMEM,
+                                         a.s>>>(static_cast<const T*>(a.z), a.idx, a.gates, a.rows, q, a.R, a.N,
+                                                static_cast<T*>(a.out));
     });
   }
   // bf16 path: Z and slots in bf16; float32 path: float32
@@ -547,10 +548,15 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
   const bool fast = d >= 64;
   const long long nang = static_cast<long long>(N) * L * (d / 2);
   if (fast) {
-    // one launch builds both tables; the phi table follows the theta table
+    // one launch builds both tables (the phi table follows the theta table)
+    // and, on the bf16 path, the bf16 copy of the base for the tensor cores
+    const TabLayout tl = make_tab_layout(d / 32, L);
+    const int tab_blocks = 2 * N * L;
+    const int exp_blocks = bf16 ? grid_for(static_cast<long long>(d) * (d / 16), 256, 1024) : 0;
     e = launch("rot_table", s, [&] {
-      rot_quads_kernel<<<2 * N * L, 256, 0, s>>>(layer->theta, layer->phi, N, d, L,
-                                                                  reinterpret_cast<float4*>(tab_t));
+      rot_quads_kernel<<<tab_blocks + exp_blocks, 256, static_cast<size_t>(d) * sizeof(float), s>>>(
+          layer->theta, layer->phi, N, d, L, tl, reinterpret_cast<float4*>(tab_t), layer->w_packed,
+          bf16 ? wbf : nullptr);
     });
   } else {
     e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->theta, nang, tab_t); });
@@ -564,11 +570,6 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
   if (e != cudaSuccess) return cuda_fail(e, "forward: pre-rotation");
 
   if (bf16 && d >= 64) {
-    const long long nw = static_cast<long long>(d) * wpr;
-    e = launch("expand_base_bf16", s, [&] {
-      expand_base_bf16_kernel<<<grid_for(nw, 256, 4096), 256, 0, s>>>(layer->w_packed, d, wpr, wbf);
-    });
-    if (e != cudaSuccess) return cuda_fail(e, "forward: expand base");
     CUtensorMap ta, tb;
     const int BN = std::min(d, 256);
     if (!make_tmap_bf16(&ta, xrot, d, R, kGemmBM) || !make_tmap_bf16(&tb, wbf, d, d, BN))
@@ -597,9 +598,9 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
   e = fast ? dispatch_fast<PostRotateFast>(d, rb) : dispatch_e<PostRotate>(d, rb);
   if (e != cudaSuccess) return cuda_fail(e, "forward: post-rotation");
 
-  const long long n4 = static_cast<long long>(T) * (d / 4);
+  const long long nv = static_cast<long long>(T) * (d / ((bf16 && fast) ? 8 : 4));
   e = launch("combine", s, [&] {
-    const int g = grid_for(n4, 256, sm_count() * 16);
+    const int g = grid_for(nv, 256, sm_count() * 16);
     if (bf16 && fast)
       combine_kernel<__nv_bfloat16, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(slot), T, k,
                                                                      d, static_cast<__nv_bfloat16*>(y));

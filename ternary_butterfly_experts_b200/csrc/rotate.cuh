@@ -214,42 +214,44 @@ __global__ __launch_bounds__(256) void post_rotate_kernel(const float* __restric
 }
 
 // y_t = sum_{j<k} slot[t*k + j] in slot order, in float32, rounded once.
+// Each thread takes 16 bytes of every slot (VEC = 16 / sizeof(Ts) columns).
 template <typename Ts, typename Tout>
 __global__ __launch_bounds__(256) void combine_kernel(const Ts* __restrict__ slot, long long T, int k, int d,
                                                       Tout* __restrict__ y) {
-  const int d4 = d / 4;
-  const long long n = T * d4;
+  constexpr int VEC = 16 / sizeof(Ts);
+  const int dv = d / VEC;
+  const long long n = T * dv;
   for (long long q = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; q < n;
        q += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long t = q / d4;
-    const int c = static_cast<int>(q % d4) * 4;
+    const long long t = q / dv;
+    const int c = static_cast<int>(q % dv) * VEC;
     const Ts* src = slot + static_cast<size_t>(t) * k * d + c;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < k; ++j) {
-      const Ts* sj = src + static_cast<size_t>(j) * d;
-      if constexpr (sizeof(Ts) == 4) {
-        const float4 s4 = __ldg(reinterpret_cast<const float4*>(sj));
-        acc[0] += s4.x;
-        acc[1] += s4.y;
-        acc[2] += s4.z;
-        acc[3] += s4.w;
-      } else {
-        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(sj));
-        const Ts* h = reinterpret_cast<const Ts*>(&raw);
+    float acc[VEC];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u] += to_f32(h[u]);
-      }
+    for (int u = 0; u < VEC; ++u) acc[u] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(j) * d));
+      const Ts* h = reinterpret_cast<const Ts*>(&raw);
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) acc[u] += to_f32(h[u]);
     }
     Tout* dst = y + static_cast<size_t>(t) * d + c;
     if constexpr (sizeof(Tout) == 4) {
-      *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+#pragma unroll
+      for (int u = 0; u < VEC; u += 4)
+        *reinterpret_cast<float4*>(dst + u) = make_float4(acc[u], acc[u + 1], acc[u + 2], acc[u + 3]);
     } else {
-      __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
-      uint2 raw;
-      raw.x = *reinterpret_cast<uint32_t*>(&lo);
-      raw.y = *reinterpret_cast<uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(dst) = raw;
+      uint32_t pk[VEC / 2];
+#pragma unroll
+      for (int u = 0; u < VEC / 2; ++u) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * u], acc[2 * u + 1]);
+        pk[u] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      if constexpr (VEC == 8) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      } else {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+      }
     }
   }
 }

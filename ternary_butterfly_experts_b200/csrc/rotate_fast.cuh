@@ -31,7 +31,8 @@ struct Geo {
   static constexpr int L = e + 5;
   static constexpr int P = e > 5 ? e : 5;
   static constexpr int D = 32 * E_;
-  static constexpr int G = E_ <= 16 ? 4 : (E_ <= 32 ? 2 : 1);  // rows per warp
+  // rows per warp: each cos/sin table load serves G rows of one expert
+  static constexpr int G = E_ <= 16 ? 4 : (E_ <= 32 ? 2 : 1);
   static constexpr int WARPS = E_ <= 64 ? 8 : 4;
 };
 
@@ -60,20 +61,67 @@ __host__ __device__ constexpr int tab_quads(int E) {
   return tab_stage_offset(E, e + 5);
 }
 
-// Quad tables: [2][N][tab_quads(E)] float4 (theta then phi).  One block per
-// (table, expert, stage), one thread per quad.
+// Offsets of each stage's quads inside one expert's table (host-computed).
+struct TabLayout {
+  int off[13];   // quad offset of stage s
+  int nq[13];    // quads of stage s
+  int total;     // quads per expert
+};
+
+inline TabLayout make_tab_layout(int E, int L) {
+  TabLayout t{};
+  for (int s = 0; s < L; ++s) {
+    t.off[s] = tab_stage_offset(E, s);
+    t.nq[s] = tab_stage_quads(E, s);
+  }
+  t.total = tab_quads(E);
+  return t;
+}
+
+// Quad tables: [2][N][total] float4 (theta then phi).  Blocks [0, 2 N L):
+// one (table, expert, stage) each, whose d/2 angles are read once
+// (coalesced), their cos and sin kept in shared memory and the quads
+// gathered from there.  Blocks from 2 N L on expand the packed ternary base
+// to bf16 (when expand_out is set), so both weight-derived inputs of the
+// forward come from one launch.
 __global__ __launch_bounds__(256) void rot_quads_kernel(const float* __restrict__ theta,
                                                         const float* __restrict__ phi, int N, int d, int L,
-                                                        float4* __restrict__ quads) {
+                                                        const TabLayout tl, float4* __restrict__ quads,
+                                                        const uint32_t* __restrict__ w_packed,
+                                                        uint16_t* __restrict__ expand_out) {
+  extern __shared__ float cs_smem[];  // [d/2] cos, then [d/2] sin
+  const int n_tab_blocks = 2 * N * L;
+  if (static_cast<int>(blockIdx.x) >= n_tab_blocks) {
+    // expand the 2-bit base: one thread per packed word (16 weights)
+    const int wpr = d / 16;
+    const long long nw = static_cast<long long>(d) * wpr;
+    for (long long q = (blockIdx.x - n_tab_blocks) * static_cast<long long>(blockDim.x) + threadIdx.x; q < nw;
+         q += static_cast<long long>(gridDim.x - n_tab_blocks) * blockDim.x) {
+      const uint32_t word = w_packed[q];
+      uint32_t pr[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        pr[m] = ternary_code_bf16((word >> (4 * m)) & 3u) | (static_cast<uint32_t>(ternary_code_bf16((word >> (4 * m + 2)) & 3u)) << 16);
+      uint4* d4 = reinterpret_cast<uint4*>(expand_out + q * 16);
+      d4[0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+      d4[1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
+    }
+    return;
+  }
   const int E = d / 32;
   const int e = L - 5;
   const int P = e > 5 ? e : 5;
   const int s = blockIdx.x % L;
   const int ex = (blockIdx.x / L) % N;
   const int which = blockIdx.x / (L * N);
-  const float* base = (which ? phi : theta) + (static_cast<size_t>(ex) * L + s) * (d / 2);
-  float4* out = quads + (static_cast<size_t>(which) * N + ex) * tab_quads(E) + tab_stage_offset(E, s);
-  const int nq = tab_stage_quads(E, s);
+  const int half = d / 2;
+  const float* base = (which ? phi : theta) + (static_cast<size_t>(ex) * L + s) * half;
+  float* cs = cs_smem;
+  float* sn = cs_smem + half;
+  for (int i = threadIdx.x; i < half; i += blockDim.x) sincosf(base[i], &sn[i], &cs[i]);
+  __syncthreads();
+  float4* out = quads + (static_cast<size_t>(which) * N + ex) * tl.total + tl.off[s];
+  const int nq = tl.nq[s];
   for (int Q = threadIdx.x; Q < nq; Q += blockDim.x) {
     const int lane = Q & 31, u = Q >> 5;
     int a, b;
@@ -97,10 +145,7 @@ __global__ __launch_bounds__(256) void rot_quads_kernel(const float* __restrict_
       a = ((qq >> (s - 4)) << s) | ((qq & ((1 << (s - 5)) - 1)) << 5) | lane;
       b = a + 32;
     }
-    float sa, ca, sb, cb;
-    sincosf(base[a], &sa, &ca);
-    sincosf(base[b], &sb, &cb);
-    out[Q] = make_float4(ca, cb, sa, sb);
+    out[Q] = make_float4(cs[a], cs[b], sn[a], sn[b]);
   }
 }
 
@@ -370,9 +415,11 @@ struct StagedCfg {
   static constexpr int ROWS = Gm::WARPS * G;
   static constexpr int THREADS = Gm::WARPS * 32;
   static constexpr size_t TAB_QUADS = tab_quads(E);
-  // expert tables kept in shared memory (18 KB each at d=512) while two CTAs
-  // still fit on an SM; larger widths read them through L1
-  static constexpr int NTAB = Gm::D <= 512 ? (sizeof(Tin) == 2 ? 2 : 1) : (Gm::D <= 1024 && sizeof(Tin) == 2 ? 1 : 0);
+  // the cos/sin tables are read through L1 (lane-interleaved, so every warp
+  // read is 512 contiguous bytes); shared memory holds the staged rows and
+  // one transpose buffer per warp
+  static constexpr int NTAB = 0;
+  static constexpr int MIN_BLOCKS = E <= 32 ? 2 : 1;
   static constexpr size_t SMEM = ROWS * Gm::D * sizeof(Tin) + NTAB * TAB_QUADS * 16 + Gm::WARPS * Gm::D * 4 +
                                  ROWS * 12 + 64;
 };
@@ -427,7 +474,7 @@ __device__ __forceinline__ void pre_rotate_rows_smem(const Tin* xs0, const float
 // xrot[p] = B(theta_e)^T x_t for bucket positions p (row r = rows[p],
 // t = r / k, e = idx[r]).
 template <int E, typename Tin, typename Tout>
-__global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS) void pre_rotate_fast_kernel(const Tin* __restrict__ x,
+__global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS, StagedCfg<E, Tin>::MIN_BLOCKS) void pre_rotate_fast_kernel(const Tin* __restrict__ x,
                                                               const int32_t* __restrict__ idx,
                                                               const int32_t* __restrict__ rows,
                                                               const float4* __restrict__ quads, long long R, int k,
@@ -546,7 +593,7 @@ __device__ __forceinline__ void post_rotate_rows_smem(const Tz* zs0, const float
 // slot[r] = g_r * B(phi_e) z_p for bucket positions p (z already scaled by
 // alpha), r = rows[p], e = idx[r].
 template <int E, typename Tz, typename Ts>
-__global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS) void post_rotate_fast_kernel(
+__global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS, StagedCfg<E, Tz>::MIN_BLOCKS) void post_rotate_fast_kernel(
     const Tz* __restrict__ z, const int32_t* __restrict__ idx, const float* __restrict__ gates,
     const int32_t* __restrict__ rows, const float4* __restrict__ quads, long long R, int N, Ts* __restrict__ slot) {
   using C = StagedCfg<E, Tz>;

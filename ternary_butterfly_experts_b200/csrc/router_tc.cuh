@@ -10,11 +10,12 @@
 // One CTA owns 128 tokens and walks the experts in chunks of BN columns.
 // Warp 0 (one lane) loads with TMA the 128x64 token tile and the three BNx64
 // weight tiles per 64-wide slice of d; warp 1 (one lane) issues the MMAs into
-// one of two TMEM accumulators; warps 2..5 read their rows' logits from TMEM
-// (warp w owns TMEM lanes 32*(w%4) ..), keep a running top-k (larger logit
+// one of two TMEM accumulators; warps 2..9 read the logits from TMEM (warp w
+// owns TMEM lanes 32*(w%4) .., warps w and w+4 take the two halves of each
+// chunk's columns), each keeping a running top-k of its half (larger logit
 // first, lower expert index on ties, NaN below every number) while the next
-// chunk is being multiplied, and finally write idx and the renormalised
-// gates.
+// chunk is being multiplied; the two partial lists of a row are merged through
+// shared memory, and the row's idx and renormalised gates are written.
 #pragma once
 #include "common.cuh"
 #include "gemm_tc.cuh"
@@ -43,11 +44,14 @@ struct RouterTcCfg {
   static constexpr uint32_t B_BYTES = BN * kGemmBK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + 3 * B_BYTES;
   static constexpr uint32_t BAR_BYTES = (2 * STAGES + 4) * 8 + 8;
-  static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr uint32_t BIAS_BYTES = BFMOE_MAX_EXPERTS * 4;             // bias staged once
+  static constexpr uint32_t MERGE_BYTES = kGemmBM * BFMOE_MAX_K * 8;        // partial top-k lists
+  static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + BIAS_BYTES + MERGE_BYTES;
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : 256));
 };
 
-constexpr int kRouterThreads = 192;
+constexpr int kRouterThreads = 320;
+constexpr int kRouterEpiWarps = 8;
 
 // Running top-K of one row in registers (K compile-time): larger logit first,
 // lower expert index first on equal logits.
@@ -93,6 +97,9 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
   uint64_t* acc_full = empty + STAGES;   // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  float* bias_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + Cfg::BAR_BYTES);
+  float* merge_v = bias_s + BFMOE_MAX_EXPERTS;                       // [128][K]
+  int* merge_i = reinterpret_cast<int*>(merge_v + kGemmBM * BFMOE_MAX_K);  // [128][K]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kGemmBM;
@@ -106,13 +113,14 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(acc_full + b, 1);
-      mbar_init(acc_empty + b, 4);  // one arrival per epilogue warp
+      mbar_init(acc_empty + b, kRouterEpiWarps);  // one arrival per epilogue warp
     }
     mbar_fence_init();
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
   }
   if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+  for (int e = threadIdx.x; e < N; e += blockDim.x) bias_s[e] = bias ? bias[e] : 0.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -176,9 +184,12 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
     return;
   }
 
-  // Epilogue (warps 2..5): one token row per thread.
+  // Epilogue (warps 2..9): one token row per thread, half of each chunk.
   const int sp = warp & 3;
-  const int row = m0 + sp * 32 + lane;
+  const int hf = (warp - 2) >> 2;  // which half of the chunk's columns
+  const int lr = sp * 32 + lane;   // row within the tile
+  const int row = m0 + lr;
+  constexpr int HALF = BN >= 64 ? BN / 2 : BN;  // columns per warp and chunk
   TopK<K> top;
   top.init();
   bool ok = true;
@@ -190,27 +201,38 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
     }
     tc_fence_after();
     const uint32_t base = tmem + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(buf * BN);
+    if (BN >= 64 || hf == 0) {
 #pragma unroll 1
-    for (int col = 0; col < BN; col += 32) {
-      const int e0 = c * BN + col;
-      float b[32];
+      for (int col = hf * HALF; col < hf * HALF + HALF; col += 32) {
+        const int e0 = c * BN + col;
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(base + static_cast<uint32_t>(col), r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int q = 0; q < 32; ++q) b[q] = (e0 + q < N) ? (bias ? __ldg(bias + e0 + q) : 0.f) : -INFINITY;
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(base + static_cast<uint32_t>(col), r);
-      tmem_wait_ld();
-#pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        float l = __uint_as_float(r[q]) + b[q];
-        if (isnan(l)) l = -INFINITY;
-        top.push(l, e0 + q < N ? e0 + q : 0x7fffffff);
+        for (int q = 0; q < 32; ++q) {
+          const int e = e0 + q;
+          float l = e < N ? __uint_as_float(r[q]) + bias_s[e] : -INFINITY;
+          if (isnan(l)) l = -INFINITY;
+          top.push(l, e < N ? e : 0x7fffffff);
+        }
       }
     }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(acc_empty + buf);
   }
-  if (ok && row < T) {
+  // merge the two halves of each row
+  if (hf == 1) {
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      merge_v[lr * BFMOE_MAX_K + j] = top.v[j];
+      merge_i[lr * BFMOE_MAX_K + j] = top.id[j];
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kRouterEpiWarps * 32) : "memory");
+  if (hf == 0 && ok && row < T) {
+#pragma unroll
+    for (int j = 0; j < K; ++j) top.push(merge_v[lr * BFMOE_MAX_K + j], merge_i[lr * BFMOE_MAX_K + j]);
     float z[K];
     float sum = 0.f;
     const bool finite_top = top.v[0] > -INFINITY;
