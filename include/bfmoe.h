@@ -120,6 +120,34 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d,
                       void* ws, size_t ws_bytes, bfmoe_stream_t stream);
 
 /*
+ * bfmoe_router_topk without a caller workspace (no counterpart on the pages:
+ * it serves callers rather than the method).  Some callers cannot allocate
+ * device memory when they call: a plug-in or kernel host that is handed only
+ * its input and output buffers, code running while the framework's allocator
+ * is locked or not reachable from the calling thread, or a runtime whose
+ * memory is planned before execution.  This call computes exactly what
+ * bfmoe_router_topk computes, using as scratch one fixed array inside the
+ * library of BFMOE_NOALLOC_SCRATCH_BYTES (every GPU that loads the library
+ * holds it until the process exits).  It allocates nothing.
+ *   - Sizes whose scratch (bfmoe_workspace_size for these sizes) exceeds the
+ *     array are rejected with BFMOE_EUNSUPPORTED before any launch.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current; make that first call before any stream capture.
+ *   - Every call shares the array: calls whose work overlaps on the GPU (on
+ *     different streams, or concurrent host threads on one device) race and
+ *     give wrong results.  Calls ordered on one stream are safe.  No part of
+ *     the array has to start at zero: each kernel writes its part before it
+ *     is read.
+ * Arguments and outputs as for bfmoe_router_topk.
+ */
+#define BFMOE_NOALLOC_SCRATCH_BYTES (32u << 20)
+int bfmoe_router_topk_noalloc(const void* x, int x_dtype, int T, int d,
+                              const float* w_gate, const float* bias, int n_experts, int k,
+                              int32_t* idx, float* gates,
+                              int32_t* counts, int32_t* offsets, int32_t* rows,
+                              bfmoe_stream_t stream);
+
+/*
  * Expert forward without forming any expert (technical summary, 2.3):
  * for every routed row, B(theta_e)^T x_t, then alpha * W_base (.), then
  * B(phi_e) (.), times the gate; the k rows of a token are summed in slot

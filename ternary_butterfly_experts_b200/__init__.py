@@ -21,6 +21,7 @@ from .capi import BFMOE_BF16, BFMOE_F32, BfmoeError
 
 __all__ = [
     "BfmoeError", "Layer", "ButterflyMoE", "bfmoe_pack_base", "bfmoe_unpack_base", "bfmoe_router_topk",
+    "bfmoe_router_topk_noalloc",
     "bfmoe_forward", "bfmoe_materialize_expert", "bfmoe_workspace_size", "bfmoe_check_device_error",
     "bfmoe_launch_count", "bfmoe_profile_enable", "bfmoe_profile_collect", "bfmoe_last_error", "workspace",
 ]
@@ -130,6 +131,33 @@ def bfmoe_router_topk(x, w_gate, bias, k: int, ws, out=None, stream=None):
         _ptr(x), _dtype_code(x), T, d, _ptr(w_gate), _ptr(bias), N, k, _ptr(idx), _ptr(gates),
         _ptr(counts), _ptr(offsets), _ptr(rows), _ptr(ws), ws.numel() if ws is not None else 0,
         _stream(stream)))
+    return out
+
+
+def bfmoe_router_topk_noalloc(x, w_gate, bias, k: int, out=None, stream=None):
+    """bfmoe_router_topk for callers that cannot allocate device memory at
+    call time: no workspace argument, the library's built-in scratch array is
+    used instead (see include/bfmoe.h for its size and sharing rules).  The
+    outputs must be provided by the caller (``out``) to allocate nothing here;
+    without ``out`` this wrapper allocates them with torch for convenience."""
+    torch = _torch()
+    _need(x, "x")
+    _need(w_gate, "w_gate", torch.float32)
+    if bias is not None:
+        _need(bias, "bias", torch.float32)
+    T, d = x.shape
+    N = w_gate.shape[0]
+    dev = x.device
+    if out is None:
+        out = (torch.empty((T, k), dtype=torch.int32, device=dev),
+               torch.empty((T, k), dtype=torch.float32, device=dev),
+               torch.empty((N,), dtype=torch.int32, device=dev),
+               torch.empty((N + 1,), dtype=torch.int32, device=dev),
+               torch.empty((T * k,), dtype=torch.int32, device=dev))
+    idx, gates, counts, offsets, rows = out
+    capi.check(capi.lib().bfmoe_router_topk_noalloc(
+        _ptr(x), _dtype_code(x), T, d, _ptr(w_gate), _ptr(bias), N, k, _ptr(idx), _ptr(gates),
+        _ptr(counts), _ptr(offsets), _ptr(rows), _stream(stream)))
     return out
 
 

@@ -23,6 +23,7 @@ BFMOE_EDEVICE_TIMEOUT = 6
 BFMOE_EDEVICE_BOUNDS = 7
 BFMOE_F32 = 0
 BFMOE_BF16 = 1
+BFMOE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 STATUS_NAMES = {0: "OK", 1: "EINVAL", 2: "ENOT_TERNARY", 3: "EUNSUPPORTED", 4: "EWORKSPACE",
                 5: "ECUDA", 6: "EDEVICE_TIMEOUT", 7: "EDEVICE_BOUNDS"}
@@ -53,6 +54,7 @@ SIGNATURES = {
     "bfmoe_pack_base": (_I, [_P, _I, _P, _P]),
     "bfmoe_unpack_base": (_I, [_P, _I, _P, _P]),
     "bfmoe_router_topk": (_I, [_P, _I, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "bfmoe_router_topk_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P]),
     "bfmoe_forward": (_I, [ctypes.POINTER(BfmoeLayer), _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bfmoe_materialize_expert": (_I, [ctypes.POINTER(BfmoeLayer), _I, _P, _P]),
     "bfmoe_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),

@@ -391,6 +391,40 @@ cudaError_t launch_router_tc(const CUtensorMap& tx, const CUtensorMap& tw, const
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Fixed scratch of bfmoe_router_topk_noalloc, for callers that cannot
+// allocate device memory.  In host code the array's name only stands for the
+// device symbol; its device address comes from cudaGetSymbolAddress, looked
+// up once per device with that device current.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[BFMOE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "router_topk_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(BFMOE_EUNSUPPORTED, "router_topk_noalloc: device %d", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "router_topk_noalloc: cudaGetSymbolAddress");
+    if (!p) return fail(BFMOE_ECUDA, "router_topk_noalloc: no device address for the scratch array");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BFMOE_OK;
+}
+
+}  // namespace
+
 // ===========================================================================
 // C ABI
 // ===========================================================================
@@ -515,6 +549,24 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
   });
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scatter");
   return ok();
+}
+
+int bfmoe_router_topk_noalloc(const void* x, int x_dtype, int T, int d, const float* w_gate, const float* bias,
+                              int n_experts, int k, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets,
+                              int32_t* rows, bfmoe_stream_t stream) {
+  int rc = check_sizes(d, n_experts, T, k);
+  if (rc) return rc;
+  if ((rc = check_dtype(x_dtype))) return rc;
+  const size_t need = make_plan(d, n_experts, T, k, x_dtype).rt_end;
+  if (need > BFMOE_NOALLOC_SCRATCH_BYTES)
+    return fail(BFMOE_EUNSUPPORTED,
+                "router_topk_noalloc: these sizes need %zu bytes of scratch; the built-in array holds %u "
+                "(use bfmoe_router_topk with a workspace)",
+                need, static_cast<unsigned>(BFMOE_NOALLOC_SCRATCH_BYTES));
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  return bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, n_experts, k, idx, gates, counts, offsets, rows, scratch,
+                           BFMOE_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, int k, const int32_t* idx,
