@@ -169,6 +169,29 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
                   void* y, void* ws, size_t ws_bytes, bfmoe_stream_t stream);
 
 /*
+ * Router and expert forward in one call: the results of bfmoe_router_topk
+ * followed by bfmoe_forward, bit for bit.  The work that depends on the
+ * weights only (the cos/sin tables of theta and phi and the bf16 copy of the
+ * base) runs on a library-owned side stream, forked from `stream` with an
+ * event and joined back before the pre-rotation, so it overlaps the router.
+ * The side stream and its two events are created once per device on first
+ * use (make that first call before any stream capture); the fork and join
+ * are stream-ordered and can be captured in a CUDA graph.  Calls from several
+ * host threads on one device share that side stream and serialise their
+ * weight-only work.
+ *   ws        device scratch of bfmoe_moe_workspace_size(...) bytes, 256-byte
+ *             aligned (the router and the tables need separate regions here)
+ * Other arguments as for bfmoe_router_topk and bfmoe_forward.
+ */
+int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T,
+                      const float* w_gate, const float* bias, int k,
+                      int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, int32_t* rows,
+                      void* y, void* ws, size_t ws_bytes, bfmoe_stream_t stream);
+
+/* Scratch bytes that bfmoe_moe_forward needs (0 for invalid sizes). */
+size_t bfmoe_moe_workspace_size(int d, int n_experts, int T, int k, int x_dtype);
+
+/*
  * Form expert e densely, alpha * B(phi_e) . W_base . B(theta_e)^T, in float32
  * (technical summary, 2.1).  For checking only.
  *   w_out     device float [d][d] (written), row = output

@@ -21,7 +21,7 @@ from .capi import BFMOE_BF16, BFMOE_F32, BfmoeError
 
 __all__ = [
     "BfmoeError", "Layer", "ButterflyMoE", "bfmoe_pack_base", "bfmoe_unpack_base", "bfmoe_router_topk",
-    "bfmoe_router_topk_noalloc",
+    "bfmoe_router_topk_noalloc", "bfmoe_moe_forward", "bfmoe_moe_workspace_size",
     "bfmoe_forward", "bfmoe_materialize_expert", "bfmoe_workspace_size", "bfmoe_check_device_error",
     "bfmoe_launch_count", "bfmoe_profile_enable", "bfmoe_profile_collect", "bfmoe_last_error", "workspace",
 ]
@@ -204,6 +204,39 @@ def bfmoe_forward(layer: Layer, x, k: int, idx, gates, offsets, rows, ws, y=None
     return y
 
 
+def bfmoe_moe_workspace_size(d: int, n_experts: int, T: int, k: int, x_dtype: int) -> int:
+    return int(capi.lib().bfmoe_moe_workspace_size(d, n_experts, T, k, x_dtype))
+
+
+def bfmoe_moe_forward(layer: Layer, x, w_gate, bias, k: int, ws, routing=None, y=None, stream=None):
+    """Router + forward in one call (weight-only work overlaps the router on a
+    side stream).  Returns (y, (idx, gates, counts, offsets, rows))."""
+    torch = _torch()
+    _need(x, "x")
+    _need(w_gate, "w_gate", torch.float32)
+    if bias is not None:
+        _need(bias, "bias", torch.float32)
+    T, d = x.shape
+    if d != layer.d:
+        raise ValueError(f"x has width {d}, layer has d={layer.d}")
+    N = layer.n_experts
+    dev = x.device
+    if routing is None:
+        routing = (torch.empty((T, k), dtype=torch.int32, device=dev),
+                   torch.empty((T, k), dtype=torch.float32, device=dev),
+                   torch.empty((N,), dtype=torch.int32, device=dev),
+                   torch.empty((N + 1,), dtype=torch.int32, device=dev),
+                   torch.empty((T * k,), dtype=torch.int32, device=dev))
+    if y is None:
+        y = torch.empty_like(x)
+    idx, gates, counts, offsets, rows = routing
+    capi.check(capi.lib().bfmoe_moe_forward(
+        ctypes.byref(layer.c), _ptr(x), _dtype_code(x), T, _ptr(w_gate), _ptr(bias), k, _ptr(idx), _ptr(gates),
+        _ptr(counts), _ptr(offsets), _ptr(rows), _ptr(y), _ptr(ws), ws.numel() if ws is not None else 0,
+        _stream(stream)))
+    return y, routing
+
+
 def bfmoe_materialize_expert(layer: Layer, e: int, out=None, stream=None):
     """alpha * B(phi_e) . W_base . B(theta_e)^T as float32 [d][d] (checking aid)."""
     torch = _torch()
@@ -244,6 +277,8 @@ class ButterflyMoE:
         dev = layer.theta.device
         N, d = layer.n_experts, layer.d
         self.ws = workspace(d, N, max_tokens, k, code, dev)
+        n = bfmoe_moe_workspace_size(d, N, max_tokens, k, code)
+        self.ws_moe = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
         self.max_tokens = max_tokens
         self.idx = torch.empty((max_tokens, k), dtype=torch.int32, device=dev)
         self.gates = torch.empty((max_tokens, k), dtype=torch.float32, device=dev)
@@ -259,13 +294,16 @@ class ButterflyMoE:
         return bfmoe_router_topk(x, self.w_gate, self.bias, self.k, self.ws, out=out, stream=stream)
 
     def __call__(self, x, y=None, stream=None):
+        """Router + forward of x (device) through bfmoe_moe_forward."""
         T = x.shape[0]
         if T > self.max_tokens:
             raise ValueError("more tokens than the buffers hold")
-        idx, gates, _, offsets, rows = self.route(x, stream)
         if y is None:
             y = self.y_dev[:T]
-        return bfmoe_forward(self.layer, x, self.k, idx, gates, offsets, rows, self.ws, y=y, stream=stream)
+        routing = (self.idx[:T], self.gates[:T], self.counts, self.offsets, self.rows[:T * self.k])
+        y, _ = bfmoe_moe_forward(self.layer, x, self.w_gate, self.bias, self.k, self.ws_moe, routing=routing, y=y,
+                                 stream=stream)
+        return y
 
     def forward_host(self, x_host, y_host, stream=None):
         """Host -> device copy, router + forward, device -> host copy."""

@@ -56,6 +56,9 @@ SIGNATURES = {
     "bfmoe_router_topk": (_I, [_P, _I, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "bfmoe_router_topk_noalloc": (_I, [_P, _I, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P]),
     "bfmoe_forward": (_I, [ctypes.POINTER(BfmoeLayer), _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "bfmoe_moe_forward": (_I, [ctypes.POINTER(BfmoeLayer), _P, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P,
+                               _SZ, _P]),
+    "bfmoe_moe_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "bfmoe_materialize_expert": (_I, [ctypes.POINTER(BfmoeLayer), _I, _P, _P]),
     "bfmoe_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "bfmoe_last_error": (ctypes.c_char_p, []),

@@ -391,6 +391,149 @@ cudaError_t launch_router_tc(const CUtensorMap& tx, const CUtensorMap& tw, const
 
 }  // namespace
 
+namespace {
+
+int check_forward_args(const bfmoe_layer* layer, const void* x, int x_dtype, int T, int k, const int32_t* idx,
+                       const float* gates, const int32_t* offsets, const int32_t* rows, const void* y) {
+  if (!layer) return fail(BFMOE_EINVAL, "forward: NULL layer");
+  int rc = check_sizes(layer->d, layer->n_experts, T, k);
+  if (rc) return rc;
+  if ((rc = check_dtype(x_dtype))) return rc;
+  if (T == 0) return BFMOE_OK;
+  if (!layer->w_packed || !layer->theta || !layer->phi) return fail(BFMOE_EINVAL, "forward: NULL layer weights");
+  if (!x || !idx || !gates || !offsets || !rows || !y) return fail(BFMOE_EINVAL, "forward: NULL pointer");
+  if (!aligned16(x) || !aligned16(y)) return fail(BFMOE_EINVAL, "forward: x and y must be 16-byte aligned");
+  return BFMOE_OK;
+}
+
+// The inputs of the forward that depend on the weights only: the cos/sin
+// tables of theta and phi and, on the bf16 path, the bf16 copy of the base.
+int build_weight_tables(const bfmoe_layer* layer, bool bf16, const Plan& p, uint8_t* W, cudaStream_t s) {
+  const int d = layer->d, N = layer->n_experts, L = ilog2(d);
+  float2* tab_t = reinterpret_cast<float2*>(W + p.tab_theta);
+  float2* tab_p = reinterpret_cast<float2*>(W + p.tab_phi);
+  uint16_t* wbf = reinterpret_cast<uint16_t*>(W + p.w_bf16);
+  const long long nang = static_cast<long long>(N) * L * (d / 2);
+  cudaError_t e;
+  if (d >= 64) {
+    // one launch builds both tables (the phi table follows the theta table)
+    // and, on the bf16 path, the bf16 copy of the base for the tensor cores
+    const TabLayout tl = make_tab_layout(d / 32, L);
+    const int tab_blocks = 2 * N;
+    const int exp_blocks = bf16 ? grid_for(static_cast<long long>(d) * (d / 16), 256, 1024) : 0;
+    const size_t tab_smem = static_cast<size_t>(L) * d * sizeof(float);  // cos and sin of one expert
+    static bool tab_attr = false;
+    if (!tab_attr) {
+      cudaFuncSetAttribute(rot_quads_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(12 * BFMOE_MAX_D * sizeof(float)));
+      tab_attr = true;
+    }
+    e = launch("rot_table", s, [&] {
+      rot_quads_kernel<<<tab_blocks + exp_blocks, 256, tab_smem, s>>>(
+          layer->theta, layer->phi, N, d, L, tl, reinterpret_cast<float4*>(tab_t), layer->w_packed,
+          bf16 ? wbf : nullptr);
+    });
+  } else {
+    e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->theta, nang, tab_t); });
+    if (e == cudaSuccess)
+      e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->phi, nang, tab_p); });
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "forward: rotation tables");
+  return BFMOE_OK;
+}
+
+// Pre-rotation, ternary product, post-rotation with gates, combine.
+int forward_body(const bfmoe_layer* layer, const void* x, bool bf16, int T, int k, const int32_t* idx,
+                 const float* gates, const int32_t* rows, void* y, const Plan& p, uint8_t* W, cudaStream_t s) {
+  const int d = layer->d, N = layer->n_experts, L = ilog2(d);
+  float2* tab_t = reinterpret_cast<float2*>(W + p.tab_theta);
+  float2* tab_p = reinterpret_cast<float2*>(W + p.tab_phi);
+  uint16_t* wbf = reinterpret_cast<uint16_t*>(W + p.w_bf16);
+  void* xrot = W + p.xrot;
+  void* z = W + p.z;
+  void* slot = W + p.slot;
+  const long long R = static_cast<long long>(T) * k;
+  const int wpr = words_per_row(d);
+  const bool fast = d >= 64;
+  cudaError_t e;
+
+  RotArgs ra{x, bf16, idx, gates, rows, tab_t, R, k, d, L, N, xrot, nullptr, s};
+  e = fast ? dispatch_fast<PreRotateFast>(d, ra) : dispatch_e<PreRotate>(d, ra);
+  if (e != cudaSuccess) return cuda_fail(e, "forward: pre-rotation");
+
+  if (bf16 && d >= 64) {
+    CUtensorMap ta, tb;
+    const int BN = std::min(d, 256);
+    if (!make_tmap_bf16(&ta, xrot, d, R, kGemmBM) || !make_tmap_bf16(&tb, wbf, d, d, BN))
+      return fail(BFMOE_ECUDA, "forward: tensor map encoding failed");
+    switch (BN) {
+      case 64: e = launch_gemm_tc<64, 8>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
+      case 128: e = launch_gemm_tc<128, 6>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
+      default: e = launch_gemm_tc<256, 4>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "forward: tensor-core GEMM");
+  } else {
+    dim3 g((R + 63) / 64, (d + 63) / 64);
+    e = launch("ternary_gemm_simt", s, [&] {
+      if (bf16)
+        ternary_gemm_simt_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(xrot),
+                                                                  layer->w_packed, wpr, R, d, layer->alpha,
+                                                                  static_cast<float*>(z));
+      else
+        ternary_gemm_simt_kernel<float><<<g, 256, 0, s>>>(static_cast<const float*>(xrot), layer->w_packed, wpr, R,
+                                                          d, layer->alpha, static_cast<float*>(z));
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "forward: SIMT ternary product");
+  }
+
+  RotArgs rb{nullptr, bf16, idx, gates, rows, tab_p, R, k, d, L, N, slot, z, s};
+  e = fast ? dispatch_fast<PostRotateFast>(d, rb) : dispatch_e<PostRotate>(d, rb);
+  if (e != cudaSuccess) return cuda_fail(e, "forward: post-rotation");
+
+  const long long nv = static_cast<long long>(T) * (d / ((bf16 && fast) ? 8 : 4));
+  e = launch("combine", s, [&] {
+    const int g = grid_for(nv, 256, sm_count() * 16);
+    if (bf16 && fast)
+      combine_kernel<__nv_bfloat16, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(slot), T, k,
+                                                                     d, static_cast<__nv_bfloat16*>(y));
+    else if (bf16)
+      combine_kernel<float, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d,
+                                                             static_cast<__nv_bfloat16*>(y));
+    else
+      combine_kernel<float, float><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d, static_cast<float*>(y));
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "forward: combine");
+  return ok();
+}
+
+// One side stream (and fork/join events) per device, created on first use,
+// for the weight-only work of bfmoe_moe_forward.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+SideStream g_side[64];
+
+int side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_forward: cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(BFMOE_EUNSUPPORTED, "moe_forward: device %d", dev);
+  std::lock_guard<std::mutex> lk(g_side_mu);
+  SideStream& ss = g_side[dev];
+  if (!ss.stream) {
+    if ((e = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_fail(e, "moe_forward: side stream");
+  }
+  *out = &ss;
+  return BFMOE_OK;
+}
+
+}  // namespace
+
 // ---------------------------------------------------------------------------
 // Fixed scratch of bfmoe_router_topk_noalloc, for callers that cannot
 // allocate device memory.  In host code the array's name only stands for the
@@ -572,98 +715,51 @@ int bfmoe_router_topk_noalloc(const void* x, int x_dtype, int T, int d, const fl
 int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, int k, const int32_t* idx,
                   const float* gates, const int32_t* offsets, const int32_t* rows, void* y, void* ws,
                   size_t ws_bytes, bfmoe_stream_t stream) {
-  if (!layer) return fail(BFMOE_EINVAL, "forward: NULL layer");
-  const int d = layer->d, N = layer->n_experts;
-  int rc = check_sizes(d, N, T, k);
-  if (rc) return rc;
-  if ((rc = check_dtype(x_dtype))) return rc;
-  if (T == 0) return ok();
-  if (!layer->w_packed || !layer->theta || !layer->phi) return fail(BFMOE_EINVAL, "forward: NULL layer weights");
-  if (!x || !idx || !gates || !offsets || !rows || !y) return fail(BFMOE_EINVAL, "forward: NULL pointer");
-  if (!aligned16(x) || !aligned16(y)) return fail(BFMOE_EINVAL, "forward: x and y must be 16-byte aligned");
-  const Plan p = make_plan(d, N, T, k, x_dtype);
+  int rc = check_forward_args(layer, x, x_dtype, T, k, idx, gates, offsets, rows, y);
+  if (rc || T == 0) return rc ? rc : ok();
+  const Plan p = make_plan(layer->d, layer->n_experts, T, k, x_dtype);
   if ((rc = check_ws(p, ws, ws_bytes, p.fwd_end))) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* W = static_cast<uint8_t*>(ws);
-  float2* tab_t = reinterpret_cast<float2*>(W + p.tab_theta);
-  float2* tab_p = reinterpret_cast<float2*>(W + p.tab_phi);
-  uint16_t* wbf = reinterpret_cast<uint16_t*>(W + p.w_bf16);
-  void* xrot = W + p.xrot;
-  void* z = W + p.z;
-  void* slot = W + p.slot;
-  const int L = ilog2(d);
-  const long long R = static_cast<long long>(T) * k;
-  const bool bf16 = x_dtype == BFMOE_BF16;
-  const int wpr = words_per_row(d);
-  cudaError_t e;
+  if ((rc = build_weight_tables(layer, x_dtype == BFMOE_BF16, p, W, s))) return rc;
+  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, s);
+}
 
-  const bool fast = d >= 64;
-  const long long nang = static_cast<long long>(N) * L * (d / 2);
-  if (fast) {
-    // one launch builds both tables (the phi table follows the theta table)
-    // and, on the bf16 path, the bf16 copy of the base for the tensor cores
-    const TabLayout tl = make_tab_layout(d / 32, L);
-    const int tab_blocks = 2 * N * L;
-    const int exp_blocks = bf16 ? grid_for(static_cast<long long>(d) * (d / 16), 256, 1024) : 0;
-    e = launch("rot_table", s, [&] {
-      rot_quads_kernel<<<tab_blocks + exp_blocks, 256, static_cast<size_t>(d) * sizeof(float), s>>>(
-          layer->theta, layer->phi, N, d, L, tl, reinterpret_cast<float4*>(tab_t), layer->w_packed,
-          bf16 ? wbf : nullptr);
-    });
-  } else {
-    e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->theta, nang, tab_t); });
-    if (e == cudaSuccess)
-      e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->phi, nang, tab_p); });
-  }
-  if (e != cudaSuccess) return cuda_fail(e, "forward: rotation tables");
+size_t bfmoe_moe_workspace_size(int d, int n_experts, int T, int k, int x_dtype) {
+  if (check_sizes(d, n_experts, T, k) != BFMOE_OK || check_dtype(x_dtype) != BFMOE_OK) return 0;
+  const Plan p = make_plan(d, n_experts, T, k, x_dtype);
+  return p.fwd_end + p.rt_end;
+}
 
-  RotArgs ra{x, bf16, idx, gates, rows, tab_t, R, k, d, L, N, xrot, nullptr, s};
-  e = fast ? dispatch_fast<PreRotateFast>(d, ra) : dispatch_e<PreRotate>(d, ra);
-  if (e != cudaSuccess) return cuda_fail(e, "forward: pre-rotation");
-
-  if (bf16 && d >= 64) {
-    CUtensorMap ta, tb;
-    const int BN = std::min(d, 256);
-    if (!make_tmap_bf16(&ta, xrot, d, R, kGemmBM) || !make_tmap_bf16(&tb, wbf, d, d, BN))
-      return fail(BFMOE_ECUDA, "forward: tensor map encoding failed");
-    switch (BN) {
-      case 64: e = launch_gemm_tc<64, 8>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
-      case 128: e = launch_gemm_tc<128, 6>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
-      default: e = launch_gemm_tc<256, 4>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
-    }
-    if (e != cudaSuccess) return cuda_fail(e, "forward: tensor-core GEMM");
-  } else {
-    dim3 g((R + 63) / 64, (d + 63) / 64);
-    e = launch("ternary_gemm_simt", s, [&] {
-      if (bf16)
-        ternary_gemm_simt_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(xrot),
-                                                                  layer->w_packed, wpr, R, d, layer->alpha,
-                                                                  static_cast<float*>(z));
-      else
-        ternary_gemm_simt_kernel<float><<<g, 256, 0, s>>>(static_cast<const float*>(xrot), layer->w_packed, wpr, R,
-                                                          d, layer->alpha, static_cast<float*>(z));
-    });
-    if (e != cudaSuccess) return cuda_fail(e, "forward: SIMT ternary product");
-  }
-
-  RotArgs rb{nullptr, bf16, idx, gates, rows, tab_p, R, k, d, L, N, slot, z, s};
-  e = fast ? dispatch_fast<PostRotateFast>(d, rb) : dispatch_e<PostRotate>(d, rb);
-  if (e != cudaSuccess) return cuda_fail(e, "forward: post-rotation");
-
-  const long long nv = static_cast<long long>(T) * (d / ((bf16 && fast) ? 8 : 4));
-  e = launch("combine", s, [&] {
-    const int g = grid_for(nv, 256, sm_count() * 16);
-    if (bf16 && fast)
-      combine_kernel<__nv_bfloat16, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(slot), T, k,
-                                                                     d, static_cast<__nv_bfloat16*>(y));
-    else if (bf16)
-      combine_kernel<float, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d,
-                                                             static_cast<__nv_bfloat16*>(y));
-    else
-      combine_kernel<float, float><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d, static_cast<float*>(y));
-  });
-  if (e != cudaSuccess) return cuda_fail(e, "forward: combine");
-  return ok();
+int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, const float* w_gate,
+                      const float* bias, int k, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets,
+                      int32_t* rows, void* y, void* ws, size_t ws_bytes, bfmoe_stream_t stream) {
+  int rc = check_forward_args(layer, x, x_dtype, T, k, idx, gates, offsets, rows, y);
+  if (rc) return rc;
+  if (!w_gate || !counts) return fail(BFMOE_EINVAL, "moe_forward: NULL pointer");
+  const int d = layer->d, N = layer->n_experts;
+  const Plan p = make_plan(d, N, T, k, x_dtype);
+  const size_t need = p.fwd_end + p.rt_end;
+  if (T > 0 && (rc = check_ws(p, ws, ws_bytes, need))) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* W = static_cast<uint8_t*>(ws);
+  if (T == 0)
+    return bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, nullptr, 0,
+                             stream);
+  // fork: the weight-derived tables build on the side stream while the router runs
+  SideStream* ss = nullptr;
+  if ((rc = side_stream(&ss))) return rc;
+  cudaError_t e = cudaEventRecord(ss->fork, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_forward: fork");
+  if ((rc = build_weight_tables(layer, x_dtype == BFMOE_BF16, p, W, ss->stream))) return rc;
+  if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return cuda_fail(e, "moe_forward: join record");
+  rc = bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, W + p.fwd_end,
+                         p.rt_end, stream);
+  // join before anything else can fail, so the side stream never outlives the call's work
+  if ((e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) return cuda_fail(e, "moe_forward: join");
+  if (rc) return rc;
+  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, s);
 }
 
 int bfmoe_materialize_expert(const bfmoe_layer* layer, int e_idx, float* w_out, bfmoe_stream_t stream) {

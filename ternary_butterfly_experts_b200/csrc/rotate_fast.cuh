@@ -78,19 +78,19 @@ inline TabLayout make_tab_layout(int E, int L) {
   return t;
 }
 
-// Quad tables: [2][N][total] float4 (theta then phi).  Blocks [0, 2 N L):
-// one (table, expert, stage) each, whose d/2 angles are read once
-// (coalesced), their cos and sin kept in shared memory and the quads
-// gathered from there.  Blocks from 2 N L on expand the packed ternary base
-// to bf16 (when expand_out is set), so both weight-derived inputs of the
-// forward come from one launch.
+// Quad tables: [2][N][total] float4 (theta then phi).  Blocks [0, 2N): one
+// (table, expert) each.  The expert's L*d/2 angles are read once (coalesced,
+// many loads in flight), their cos and sin kept in shared memory, then every
+// stage's quads are gathered from there.  Blocks from 2N on expand the packed
+// ternary base to bf16 (when expand_out is set), so both weight-derived
+// inputs of the forward come from one launch.
 __global__ __launch_bounds__(256) void rot_quads_kernel(const float* __restrict__ theta,
                                                         const float* __restrict__ phi, int N, int d, int L,
                                                         const TabLayout tl, float4* __restrict__ quads,
                                                         const uint32_t* __restrict__ w_packed,
                                                         uint16_t* __restrict__ expand_out) {
-  extern __shared__ float cs_smem[];  // [d/2] cos, then [d/2] sin
-  const int n_tab_blocks = 2 * N * L;
+  extern __shared__ float cs_smem[];  // [L*d/2] cos, then [L*d/2] sin
+  const int n_tab_blocks = 2 * N;
   if (static_cast<int>(blockIdx.x) >= n_tab_blocks) {
     // expand the 2-bit base: one thread per packed word (16 weights)
     const int wpr = d / 16;
@@ -101,7 +101,8 @@ __global__ __launch_bounds__(256) void rot_quads_kernel(const float* __restrict_
       uint32_t pr[8];
 #pragma unroll
       for (int m = 0; m < 8; ++m)
-        pr[m] = ternary_code_bf16((word >> (4 * m)) & 3u) | (static_cast<uint32_t>(ternary_code_bf16((word >> (4 * m + 2)) & 3u)) << 16);
+        pr[m] = ternary_code_bf16((word >> (4 * m)) & 3u) |
+                (static_cast<uint32_t>(ternary_code_bf16((word >> (4 * m + 2)) & 3u)) << 16);
       uint4* d4 = reinterpret_cast<uint4*>(expand_out + q * 16);
       d4[0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
       d4[1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
@@ -111,41 +112,46 @@ __global__ __launch_bounds__(256) void rot_quads_kernel(const float* __restrict_
   const int E = d / 32;
   const int e = L - 5;
   const int P = e > 5 ? e : 5;
-  const int s = blockIdx.x % L;
-  const int ex = (blockIdx.x / L) % N;
-  const int which = blockIdx.x / (L * N);
+  const int ex = blockIdx.x % N;
+  const int which = blockIdx.x / N;
   const int half = d / 2;
-  const float* base = (which ? phi : theta) + (static_cast<size_t>(ex) * L + s) * half;
+  const int nang = L * half;
+  const float* base = (which ? phi : theta) + static_cast<size_t>(ex) * nang;
   float* cs = cs_smem;
-  float* sn = cs_smem + half;
-  for (int i = threadIdx.x; i < half; i += blockDim.x) sincosf(base[i], &sn[i], &cs[i]);
+  float* sn = cs_smem + nang;
+  for (int i = threadIdx.x; i < nang; i += blockDim.x) sincosf(base[i], &sn[i], &cs[i]);
   __syncthreads();
-  float4* out = quads + (static_cast<size_t>(which) * N + ex) * tl.total + tl.off[s];
-  const int nq = tl.nq[s];
-  for (int Q = threadIdx.x; Q < nq; Q += blockDim.x) {
-    const int lane = Q & 31, u = Q >> 5;
-    int a, b;
-    if (s < P && s >= e) {  // cross-lane: rotations base + 2u, base + 2u + 1
-      const int m = 1 << (s - e);
-      const int i_lo = (lane & ~m) * E;
-      a = rot_index(i_lo, s) + 2 * u;
-      b = a + 1;
-    } else if (s == 0) {  // layout 1, pairs (q, q+1): rotations l*E/2 + 2u, +1
-      a = lane * (E / 2) + 2 * u;
-      b = E >= 4 ? a + 1 : a;
-    } else if (s < P) {  // layout 1 in registers: the u-th even q with bit s clear
-      const int q = ((u >> (s - 1)) << (s + 1)) | ((u & ((1 << (s - 1)) - 1)) << 1);
-      a = lane * (E / 2) + ((q >> (s + 1)) << s) + (q & ((1 << s) - 1));
-      b = a + 1;
-    } else if (s == 5) {  // layout 2, stage 5: natural order
-      a = 2 * Q;
-      b = a + 1;
-    } else {  // layout 2, s >= 6: lane l's registers q and q+1 (b = a + 32)
-      const int qq = ((u >> (s - 6)) << (s - 4)) | ((u & ((1 << (s - 6)) - 1)) << 1);
-      a = ((qq >> (s - 4)) << s) | ((qq & ((1 << (s - 5)) - 1)) << 5) | lane;
-      b = a + 32;
+  float4* out0 = quads + (static_cast<size_t>(which) * N + ex) * tl.total;
+  for (int s = 0; s < L; ++s) {
+    const float* cst = cs + s * half;
+    const float* snt = sn + s * half;
+    float4* out = out0 + tl.off[s];
+    const int nq = tl.nq[s];
+    for (int Q = threadIdx.x; Q < nq; Q += blockDim.x) {
+      const int lane = Q & 31, u = Q >> 5;
+      int a, b;
+      if (s < P && s >= e) {  // cross-lane: rotations base + 2u, base + 2u + 1
+        const int m = 1 << (s - e);
+        const int i_lo = (lane & ~m) * E;
+        a = rot_index(i_lo, s) + 2 * u;
+        b = a + 1;
+      } else if (s == 0) {  // layout 1, pairs (q, q+1): rotations l*E/2 + 2u, +1
+        a = lane * (E / 2) + 2 * u;
+        b = E >= 4 ? a + 1 : a;
+      } else if (s < P) {  // layout 1 in registers: the u-th even q with bit s clear
+        const int q = ((u >> (s - 1)) << (s + 1)) | ((u & ((1 << (s - 1)) - 1)) << 1);
+        a = lane * (E / 2) + ((q >> (s + 1)) << s) + (q & ((1 << s) - 1));
+        b = a + 1;
+      } else if (s == 5) {  // layout 2, stage 5: natural order
+        a = 2 * Q;
+        b = a + 1;
+      } else {  // layout 2, s >= 6: lane l's registers q and q+1 (b = a + 32)
+        const int qq = ((u >> (s - 6)) << (s - 4)) | ((u & ((1 << (s - 6)) - 1)) << 1);
+        a = ((qq >> (s - 4)) << s) | ((qq & ((1 << (s - 5)) - 1)) << 5) | lane;
+        b = a + 32;
+      }
+      out[Q] = make_float4(cst[a], cst[b], snt[a], snt[b]);
     }
-    out[Q] = make_float4(cs[a], cs[b], sn[a], sn[b]);
   }
 }
 
@@ -389,13 +395,15 @@ __device__ __forceinline__ void to_layout1(float (&r)[E], float* buf, int lane) 
   __syncwarp();
 }
 
-// ---- kernels: rows and cos/sin tables staged in shared memory ------------------
+// ---- kernels: each warp stages its own rows in shared memory --------------------
 //
-// A CTA takes ROWS = WARPS * G consecutive bucket positions.  It first copies
-// the gathered input rows and the cos/sin tables of the first and last expert
-// of its range (bucket order sorts rows by expert) into shared memory with
-// cp.async, so the global-load latency of one CTA overlaps the arithmetic of
-// the others on the SM; warp w then rotates rows [w*G, w*G + G).
+// Warp w of CTA b takes G consecutive bucket positions.  Lanes 0..G-1 read
+// their rows' ids and experts; the warp copies its G gathered rows into its
+// own slice of shared memory with cp.async and waits only for its own copies,
+// so there is no CTA-wide barrier: one warp's load latency overlaps the
+// arithmetic of the others.  A group whose rows share one expert is rotated
+// together (G rows per cos/sin load, tables read through L1); a mixed group
+// row by row.
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
@@ -404,24 +412,21 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-// 16-byte chunk c of a staged float32 row sits at chunk c ^ ((c >> 3) & 7):
-// layout-1 float4 reads of 8 lanes then hit 8 different bank groups.
+// 16-byte chunk c of a staged row sits at chunk c ^ ((c >> 3) & 7): layout-1
+// reads of 8 lanes then hit 8 different bank groups.
 __device__ __forceinline__ int chunk_swz(int c) { return c ^ ((c >> 3) & 7); }
 
 template <int E, typename Tin>
 struct StagedCfg {
   using Gm = Geo<E>;
   static constexpr int G = Gm::G;
-  static constexpr int ROWS = Gm::WARPS * G;
   static constexpr int THREADS = Gm::WARPS * 32;
   static constexpr size_t TAB_QUADS = tab_quads(E);
-  // the cos/sin tables are read through L1 (lane-interleaved, so every warp
-  // read is 512 contiguous bytes); shared memory holds the staged rows and
-  // one transpose buffer per warp
-  static constexpr int NTAB = 0;
   static constexpr int MIN_BLOCKS = E <= 32 ? 2 : 1;
-  static constexpr size_t SMEM = ROWS * Gm::D * sizeof(Tin) + NTAB * TAB_QUADS * 16 + Gm::WARPS * Gm::D * 4 +
-                                 ROWS * 12 + 64;
+  // per warp: its G staged rows and one float32 transpose buffer
+  static constexpr size_t WARP_BYTES = G * Gm::D * sizeof(Tin) + Gm::D * 4;
+  static constexpr size_t SMEM = Gm::WARPS * WARP_BYTES;
+  static constexpr int ROWS = Gm::WARPS * G;  // bucket positions per CTA
 };
 
 struct RowMeta {
@@ -430,28 +435,24 @@ struct RowMeta {
   float gate;
 };
 
-// Stage the tables of the first and last expert of the CTA's range; returns
-// where each row's table lives (shared memory when staged, else global).
-template <class C>
-__device__ __forceinline__ const float4* table_for(int e, int ea, int eb, const float4* smem_tab,
-                                                   const float4* __restrict__ quads) {
-  if (C::NTAB >= 1 && e == ea) return smem_tab;
-  if (C::NTAB >= 2 && e == eb) return smem_tab + C::TAB_QUADS;
-  return quads + static_cast<size_t>(e) * C::TAB_QUADS;
+// Lane g < G reads bucket position p0 + g: its row, expert and gate.
+__device__ __forceinline__ RowMeta fetch_row_meta(const int32_t* __restrict__ rows, const int32_t* __restrict__ idx,
+                                                  const float* __restrict__ gates, long long p, long long R, int N) {
+  RowMeta m{-1, -1, 0.f};
+  if (p < R) {
+    const int r = rows[p];
+    if (r >= 0 && r < R) {
+      const int e = idx[r];
+      if (e >= 0 && e < N) m = RowMeta{r, e, gates ? gates[r] : 0.f};
+    }
+    if (m.ex < 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
+  }
+  return m;
 }
 
-template <class C>
-__device__ __forceinline__ void stage_tables(int ea, int eb, float4* smem_tab, const float4* __restrict__ quads) {
-  if constexpr (C::NTAB >= 1) {
-    if (ea >= 0)
-      for (size_t i = threadIdx.x; i < C::TAB_QUADS; i += blockDim.x)
-        cp_async16(smem_tab + i, quads + static_cast<size_t>(ea) * C::TAB_QUADS + i);
-  }
-  if constexpr (C::NTAB >= 2) {
-    if (eb >= 0 && eb != ea)
-      for (size_t i = threadIdx.x; i < C::TAB_QUADS; i += blockDim.x)
-        cp_async16(smem_tab + C::TAB_QUADS + i, quads + static_cast<size_t>(eb) * C::TAB_QUADS + i);
-  }
+__device__ __forceinline__ RowMeta shfl_meta(const RowMeta& m, int src) {
+  return RowMeta{__shfl_sync(FULL_MASK, m.row, src), __shfl_sync(FULL_MASK, m.ex, src),
+                 __shfl_sync(FULL_MASK, m.gate, src)};
 }
 
 template <class Gm, int G, typename Tin, typename Tout>
@@ -474,72 +475,44 @@ __device__ __forceinline__ void pre_rotate_rows_smem(const Tin* xs0, const float
 // xrot[p] = B(theta_e)^T x_t for bucket positions p (row r = rows[p],
 // t = r / k, e = idx[r]).
 template <int E, typename Tin, typename Tout>
-__global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS, StagedCfg<E, Tin>::MIN_BLOCKS) void pre_rotate_fast_kernel(const Tin* __restrict__ x,
-                                                              const int32_t* __restrict__ idx,
-                                                              const int32_t* __restrict__ rows,
-                                                              const float4* __restrict__ quads, long long R, int k,
-                                                              int N, Tout* __restrict__ xrot) {
+__global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS, StagedCfg<E, Tin>::MIN_BLOCKS) void pre_rotate_fast_kernel(
+    const Tin* __restrict__ x, const int32_t* __restrict__ idx, const int32_t* __restrict__ rows,
+    const float4* __restrict__ quads, long long R, int k, int N, Tout* __restrict__ xrot) {
   using C = StagedCfg<E, Tin>;
   using Gm = typename C::Gm;
-  constexpr int G = C::G, ROWS = C::ROWS, D = Gm::D;
+  constexpr int G = C::G, D = Gm::D;
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  Tin* xs = reinterpret_cast<Tin*>(smem_raw);
-  float4* tab = reinterpret_cast<float4*>(smem_raw + ROWS * D * sizeof(Tin));
-  float* tbuf = reinterpret_cast<float*>(smem_raw + ROWS * D * sizeof(Tin) + C::NTAB * C::TAB_QUADS * 16);
-  RowMeta* meta = reinterpret_cast<RowMeta*>(tbuf + Gm::WARPS * D);
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const long long p0 = static_cast<long long>(blockIdx.x) * ROWS;
+  const long long p0 = (static_cast<long long>(blockIdx.x) * Gm::WARPS + w) * G;
+  if (p0 >= R) return;
+  uint8_t* wbase = smem_raw + w * C::WARP_BYTES;
+  Tin* xs = reinterpret_cast<Tin*>(wbase);
+  float* buf = reinterpret_cast<float*>(wbase + G * D * sizeof(Tin));
 
-  if (threadIdx.x < ROWS) {
-    const long long p = p0 + threadIdx.x;
-    RowMeta m{-1, -1, 0.f};
-    if (p < R) {
-      const int r = rows[p];
-      if (r >= 0 && r < R) {
-        const int e = idx[r];
-        if (e >= 0 && e < N) m = RowMeta{r, e, 0.f};
-      }
-      if (m.ex < 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
-    }
-    meta[threadIdx.x] = m;
-  }
-  __syncthreads();
-  // first and last expert of the range (rows are sorted by expert)
-  static_assert(ROWS <= 32, "one warp ballot covers the range");
-  const int my_ex = lane < ROWS ? meta[lane].ex : -1;
-  const unsigned vm = __ballot_sync(FULL_MASK, my_ex >= 0);
-  const int ea = vm ? __shfl_sync(FULL_MASK, my_ex, __ffs(vm) - 1) : -1;
-  const int eb = vm ? __shfl_sync(FULL_MASK, my_ex, 31 - __clz(vm)) : -1;
-  // gathered input rows (invalid rows read token 0; their output is zeroed)
+  const RowMeta mine = lane < G ? fetch_row_meta(rows, idx, nullptr, p0 + lane, R, N) : RowMeta{-1, -1, 0.f};
+  const int my_tok = mine.row >= 0 ? mine.row / k : 0;  // invalid rows read token 0; output zeroed
   constexpr int CH = D * sizeof(Tin) / 16;
-  for (int i = threadIdx.x; i < ROWS * CH; i += blockDim.x) {
-    const int rr = i / CH, c = i % CH;
-    const int rid = meta[rr].row;
-    const int t = rid >= 0 ? rid / k : 0;
-    cp_async16(reinterpret_cast<uint8_t*>(xs) + static_cast<size_t>(rr) * D * sizeof(Tin) + c * 16,
+  for (int i = lane; i < G * CH; i += 32) {
+    const int g = i / CH, c = i % CH;
+    const int t = __shfl_sync(__activemask(), my_tok, g);
+    cp_async16(reinterpret_cast<uint8_t*>(xs) + static_cast<size_t>(g) * D * sizeof(Tin) + c * 16,
                reinterpret_cast<const uint8_t*>(x + static_cast<size_t>(t) * D) + c * 16);
   }
-  stage_tables<C>(ea, eb, tab, quads);
   cp_async_wait_all();
-  __syncthreads();
+  __syncwarp();
 
-  float* buf = tbuf + w * D;
-  const int r0 = w * G;
-  if (p0 + r0 >= R) return;
-  bool same = p0 + r0 + G <= R;
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-    if (meta[r0 + g].ex < 0 || meta[r0 + g].ex != meta[r0].ex) same = false;
-  if (same) {
-    pre_rotate_rows_smem<Gm, G, Tin, Tout>(xs + r0 * D, table_for<C>(meta[r0].ex, ea, eb, tab, quads),
-                                           xrot + (p0 + r0) * D, buf, lane);
+  const int e0 = __shfl_sync(FULL_MASK, mine.ex, 0);
+  const unsigned same = __ballot_sync(FULL_MASK, lane < G && mine.ex >= 0 && mine.ex == e0);
+  if (same == (1u << G) - 1u && p0 + G <= R) {
+    pre_rotate_rows_smem<Gm, G, Tin, Tout>(xs, quads + static_cast<size_t>(e0) * C::TAB_QUADS, xrot + p0 * D, buf,
+                                           lane);
     return;
   }
 #pragma unroll 1
   for (int g = 0; g < G; ++g) {
-    const long long p = p0 + r0 + g;
+    const long long p = p0 + g;
     if (p >= R) break;
-    const int e = meta[r0 + g].ex;
+    const int e = __shfl_sync(FULL_MASK, mine.ex, g);
     if (e < 0) {
       float z[E];
 #pragma unroll
@@ -547,7 +520,7 @@ __global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS, StagedCfg<E, Tin>::MIN_
       store_row<E, Tout>(xrot + p * D + lane * E, z, true);
       continue;
     }
-    pre_rotate_rows_smem<Gm, 1, Tin, Tout>(xs + (r0 + g) * D, table_for<C>(e, ea, eb, tab, quads), xrot + p * D,
+    pre_rotate_rows_smem<Gm, 1, Tin, Tout>(xs + g * D, quads + static_cast<size_t>(e) * C::TAB_QUADS, xrot + p * D,
                                            buf, lane);
   }
 }
@@ -598,66 +571,42 @@ __global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS, StagedCfg<E, Tz>::MIN_BL
     const int32_t* __restrict__ rows, const float4* __restrict__ quads, long long R, int N, Ts* __restrict__ slot) {
   using C = StagedCfg<E, Tz>;
   using Gm = typename C::Gm;
-  constexpr int G = C::G, ROWS = C::ROWS, D = Gm::D;
+  constexpr int G = C::G, D = Gm::D;
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  Tz* zs = reinterpret_cast<Tz*>(smem_raw);
-  float4* tab = reinterpret_cast<float4*>(smem_raw + ROWS * D * sizeof(Tz));
-  float* tbuf = reinterpret_cast<float*>(smem_raw + ROWS * D * sizeof(Tz) + C::NTAB * C::TAB_QUADS * 16);
-  RowMeta* meta = reinterpret_cast<RowMeta*>(tbuf + Gm::WARPS * D);
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const long long p0 = static_cast<long long>(blockIdx.x) * ROWS;
+  const long long p0 = (static_cast<long long>(blockIdx.x) * Gm::WARPS + w) * G;
+  if (p0 >= R) return;
+  uint8_t* wbase = smem_raw + w * C::WARP_BYTES;
+  Tz* zs = reinterpret_cast<Tz*>(wbase);
+  float* buf = reinterpret_cast<float*>(wbase + G * D * sizeof(Tz));
 
-  if (threadIdx.x < ROWS) {
-    const long long p = p0 + threadIdx.x;
-    RowMeta m{-1, -1, 0.f};
-    if (p < R) {
-      const int r = rows[p];
-      if (r >= 0 && r < R) {
-        const int e = idx[r];
-        if (e >= 0 && e < N) m = RowMeta{r, e, gates[r]};
-      }
-      if (m.ex < 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
-    }
-    meta[threadIdx.x] = m;
-  }
-  __syncthreads();
-  // first and last expert of the range (rows are sorted by expert)
-  static_assert(ROWS <= 32, "one warp ballot covers the range");
-  const int my_ex = lane < ROWS ? meta[lane].ex : -1;
-  const unsigned vm = __ballot_sync(FULL_MASK, my_ex >= 0);
-  const int ea = vm ? __shfl_sync(FULL_MASK, my_ex, __ffs(vm) - 1) : -1;
-  const int eb = vm ? __shfl_sync(FULL_MASK, my_ex, 31 - __clz(vm)) : -1;
+  const RowMeta mine = lane < G ? fetch_row_meta(rows, idx, gates, p0 + lane, R, N) : RowMeta{-1, -1, 0.f};
   constexpr int CH = D * sizeof(Tz) / 16;  // 16-byte chunks per row
-  for (int i = threadIdx.x; i < ROWS * CH; i += blockDim.x) {
-    const int rr = i / CH, c = i % CH;
-    const long long p = p0 + rr < R ? p0 + rr : R - 1;
-    cp_async16(reinterpret_cast<uint8_t*>(zs) + static_cast<size_t>(rr) * D * sizeof(Tz) + 16 * chunk_swz(c),
+  for (int i = lane; i < G * CH; i += 32) {
+    const int g = i / CH, c = i % CH;
+    const long long p = p0 + g < R ? p0 + g : R - 1;
+    cp_async16(reinterpret_cast<uint8_t*>(zs) + static_cast<size_t>(g) * D * sizeof(Tz) + 16 * chunk_swz(c),
                reinterpret_cast<const uint8_t*>(z + p * D) + 16 * c);
   }
-  stage_tables<C>(ea, eb, tab, quads);
   cp_async_wait_all();
-  __syncthreads();
+  __syncwarp();
 
-  float* buf = tbuf + w * D;
-  const int r0 = w * G;
-  if (p0 + r0 >= R) return;
-  bool same = p0 + r0 + G <= R;
+  const int e0 = __shfl_sync(FULL_MASK, mine.ex, 0);
+  const unsigned same = __ballot_sync(FULL_MASK, lane < G && mine.ex >= 0 && mine.ex == e0);
+  if (same == (1u << G) - 1u && p0 + G <= R) {
+    RowMeta m[G];
 #pragma unroll
-  for (int g = 0; g < G; ++g)
-    if (meta[r0 + g].ex < 0 || meta[r0 + g].ex != meta[r0].ex) same = false;
-  if (same) {
-    post_rotate_rows_smem<Gm, G, Tz, Ts>(zs + r0 * D, table_for<C>(meta[r0].ex, ea, eb, tab, quads), meta + r0,
-                                         slot, buf, lane);
+    for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, g);
+    post_rotate_rows_smem<Gm, G, Tz, Ts>(zs, quads + static_cast<size_t>(e0) * C::TAB_QUADS, m, slot, buf, lane);
     return;
   }
 #pragma unroll 1
   for (int g = 0; g < G; ++g) {
-    const long long p = p0 + r0 + g;
-    if (p >= R) break;
-    const int e = meta[r0 + g].ex;
-    if (e < 0) continue;
-    post_rotate_rows_smem<Gm, 1, Tz, Ts>(zs + (r0 + g) * D, table_for<C>(e, ea, eb, tab, quads), meta + r0 + g,
-                                         slot, buf, lane);
+    if (p0 + g >= R) break;
+    const RowMeta m1[1] = {shfl_meta(mine, g)};
+    if (m1[0].ex < 0) continue;
+    post_rotate_rows_smem<Gm, 1, Tz, Ts>(zs + g * D, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS, m1, slot,
+                                         buf, lane);
   }
 }
 

@@ -194,3 +194,46 @@ def test_bad_routing_is_reported_not_faulted():
         m.bfmoe_check_device_error()
     assert ei.value.status == 7
     m.bfmoe_check_device_error()  # cleared
+
+
+# -- the combined call -------------------------------------------------------------
+
+@pytest.mark.parametrize("d,N,k,T,dt", [(512, 64, 2, 777, "bf16"), (64, 8, 2, 256, "f32"), (32, 4, 3, 50, "bf16")])
+def test_moe_forward_equals_router_then_forward(d, N, k, T, dt):
+    m = B()
+    wl = W.custom("mf", d=d, n_experts=N, k=k, tokens=T, dtype=dt, bias_var=0.5)
+    inp = W.generate(wl, seed=d + T)
+    gpu = run_cuda(inp)
+    x = gpu["x"]
+    wg = torch.from_numpy(inp.w_gate).cuda()
+    bias = torch.from_numpy(inp.bias).cuda()
+    code = m.BFMOE_BF16 if dt == "bf16" else m.BFMOE_F32
+    ws = torch.empty(m.bfmoe_moe_workspace_size(d, N, T, k, code), dtype=torch.uint8, device="cuda")
+    for _ in range(2):  # the second call reuses the side stream and events
+        y, (idx, gates, counts, offsets, rows) = m.bfmoe_moe_forward(gpu["layer"], x, wg, bias, k, ws)
+        m.bfmoe_check_device_error()
+        assert np.array_equal(idx.cpu().numpy(), gpu["idx"])
+        assert np.array_equal(rows.cpu().numpy(), gpu["rows"])
+        assert np.array_equal(y.float().cpu().numpy().astype(np.float64), gpu["y"])
+
+
+def test_moe_forward_in_a_cuda_graph():
+    m = B()
+    wl = W.custom("mg", d=512, n_experts=32, k=2, tokens=300, dtype="bf16", bias_var=0.5)
+    inp = W.generate(wl, seed=5)
+    gpu = run_cuda(inp)
+    model = m.ButterflyMoE(gpu["layer"], torch.from_numpy(inp.w_gate).cuda(),
+                           torch.from_numpy(inp.bias).cuda(), 2, 300, torch.bfloat16)
+    x = gpu["x"]
+    y = torch.empty_like(x)
+    model(x, y=y)  # first call creates the side stream before capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        model(x, y=y)
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    m.bfmoe_check_device_error()
+    assert np.array_equal(y.float().cpu().numpy().astype(np.float64), gpu["y"])
+    del g
