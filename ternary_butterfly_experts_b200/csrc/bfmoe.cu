@@ -153,7 +153,7 @@ Plan make_plan(int d, int N, long long T, int k, int xdt) {
   p.slot = take(static_cast<size_t>(R) * d * inter);
   p.fwd_end = off;
   off = 0;
-  const long long nchunks = (R + kBucketChunk - 1) / kBucketChunk;
+  const long long nchunks = (R + bucket_chunk(k) - 1) / bucket_chunk(k);
   p.logits = take(static_cast<size_t>(T) * N * 4);
   p.chunk_counts = take(static_cast<size_t>(std::max(1LL, nchunks)) * N * 4);
   p.totals = take(static_cast<size_t>(N) * 4);
@@ -275,32 +275,35 @@ struct PostRotate {
   }
 };
 
+// CTAs of `kernel` that stay resident on the whole device (at least one per SM).
+template <typename K>
+int resident_ctas(K kernel, int threads, size_t smem) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  return per_sm * sm_count();
+}
+
 template <int E>
 struct PreRotateFast {
-  static cudaError_t run(const RotArgs& a) {
-    using Cb = StagedCfg<E, __nv_bfloat16>;
-    using Cf = StagedCfg<E, float>;
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(pre_rotate_fast_kernel<E, __nv_bfloat16, __nv_bfloat16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cb::SMEM));
-      cudaFuncSetAttribute(pre_rotate_fast_kernel<E, float, float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(Cf::SMEM));
-      attr = true;
+  template <typename T>
+  static cudaError_t go(const RotArgs& a) {
+    using C = StagedCfg<E, T>;
+    auto kern = pre_rotate_fast_kernel<E, T, T>;
+    static int resident = 0;
+    if (resident == 0) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
+      resident = resident_ctas(kern, C::THREADS, C::SMEM);
     }
-    const float4* q = reinterpret_cast<const float4*>(a.cs);
+    const int grid = staged_grid<E, T>((a.R + C::G - 1) / C::G, resident);
     return launch("pre_rotate", a.s, [&] {
-      if (a.bf16)
-        pre_rotate_fast_kernel<E, __nv_bfloat16, __nv_bfloat16>
-            <<<static_cast<int>((a.R + Cb::ROWS - 1) / Cb::ROWS), Cb::THREADS, Cb::SMEM, a.s>>>(
-                static_cast<const __nv_bfloat16*>(a.x), a.idx, a.rows, q, a.R, a.k, a.N,
-                static_cast<__nv_bfloat16*>(a.out));
-      else
-        pre_rotate_fast_kernel<E, float, float>
-            <<<static_cast<int>((a.R + Cf::ROWS - 1) / Cf::ROWS), Cf::THREADS, Cf::SMEM, a.s>>>(
-                static_cast<const float*>(a.x), a.idx, a.rows, q, a.R, a.k, a.N, static_cast<float*>(a.out));
+      kern<<<grid, C::THREADS, C::SMEM, a.s>>>(static_cast<const T*>(a.x), a.idx, a.rows,
+                                               reinterpret_cast<const float4*>(a.cs), a.R, a.k, a.N,
+                                               static_cast<T*>(a.out));
     });
   }
+  // bf16 path: x and X_rot in bf16; float32 path: float32
+  static cudaError_t run(const RotArgs& a) { return a.bf16 ? go<__nv_bfloat16>(a) : go<float>(a); }
 };
 
 template <int E>
@@ -308,17 +311,17 @@ struct PostRotateFast {
   template <typename T>
   static cudaError_t go(const RotArgs& a) {
     using C = StagedCfg<E, T>;
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(post_rotate_fast_kernel<E, T, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(C::SMEM));
-      attr = true;
+    auto kern = post_rotate_fast_kernel<E, T, T>;
+    static int resident = 0;
+    if (resident == 0) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
+      resident = resident_ctas(kern, C::THREADS, C::SMEM);
     }
-    const float4* q = reinterpret_cast<const float4*>(a.cs);
+    const int grid = staged_grid<E, T>((a.R + C::G - 1) / C::G, resident);
     return launch("post_rotate", a.s, [&] {
-      post_rotate_fast_kernel<E, T, T><<<static_cast<int>((a.R + C::ROWS - 1) / C::ROWS), C::THREADS, C::SMEM,
-                                         a.s>>>(static_cast<const T*>(a.z), a.idx, a.gates, a.rows, q, a.R, a.N,
-                                                static_cast<T*>(a.out));
+      kern<<<grid, C::THREADS, C::SMEM, a.s>>>(static_cast<const T*>(a.z), a.idx, a.gates, a.rows,
+                                               reinterpret_cast<const float4*>(a.cs), a.R, a.N,
+                                               static_cast<T*>(a.out));
     });
   }
   // bf16 path: Z and slots in bf16; float32 path: float32
@@ -340,8 +343,8 @@ cudaError_t dispatch_fast(int d, A&&... a) {
 }
 
 template <int BN, int STAGES>
-cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, __nv_bfloat16* z, int R, int d, float alpha,
-                           cudaStream_t s) {
+cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tbh, __nv_bfloat16* z,
+                           int R, int d, float alpha, cudaStream_t s) {
   using Cfg = GemmTcCfg<BN, STAGES>;
   static bool attr = false;
   if (!attr) {
@@ -353,13 +356,13 @@ cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, __nv_bf
   const long long tiles = static_cast<long long>((R + kGemmBM - 1) / kGemmBM) * (d / BN);
   const int grid = static_cast<int>(std::min<long long>(tiles, sm_count()));
   return launch("ternary_gemm_tc", s, [&] {
-    ternary_gemm_tc_kernel<BN, STAGES><<<grid, kGemmThreads, Cfg::SMEM_BYTES, s>>>(ta, tb, z, R, d, alpha);
+    ternary_gemm_tc_kernel<BN, STAGES><<<grid, kGemmThreads, Cfg::SMEM_BYTES, s>>>(ta, tb, tbh, z, R, d, alpha);
   });
 }
 
 template <int BN, int STAGES, int K>
 cudaError_t launch_router_tc_k(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
-                               int32_t* idx, float* gates, cudaStream_t s) {
+                               int32_t* idx, float* gates, int32_t* cc, cudaStream_t s) {
   using Cfg = RouterTcCfg<BN, STAGES>;
   static bool attr = false;
   if (!attr) {
@@ -370,22 +373,22 @@ cudaError_t launch_router_tc_k(const CUtensorMap& tx, const CUtensorMap& tw, con
   }
   const int grid = (T + kGemmBM - 1) / kGemmBM;
   return launch("router_tc", s, [&] {
-    router_tc_kernel<BN, STAGES, K><<<grid, kRouterThreads, Cfg::SMEM_BYTES, s>>>(tx, tw, bias, T, d, N, idx, gates);
+    router_tc_kernel<BN, STAGES, K><<<grid, kRouterThreads, Cfg::SMEM_BYTES, s>>>(tx, tw, bias, T, d, N, idx, gates, cc);
   });
 }
 
 template <int BN, int STAGES>
 cudaError_t launch_router_tc(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
-                             int k, int32_t* idx, float* gates, cudaStream_t s) {
+                             int k, int32_t* idx, float* gates, int32_t* cc, cudaStream_t s) {
   switch (k) {
-    case 1: return launch_router_tc_k<BN, STAGES, 1>(tx, tw, bias, T, d, N, idx, gates, s);
-    case 2: return launch_router_tc_k<BN, STAGES, 2>(tx, tw, bias, T, d, N, idx, gates, s);
-    case 3: return launch_router_tc_k<BN, STAGES, 3>(tx, tw, bias, T, d, N, idx, gates, s);
-    case 4: return launch_router_tc_k<BN, STAGES, 4>(tx, tw, bias, T, d, N, idx, gates, s);
-    case 5: return launch_router_tc_k<BN, STAGES, 5>(tx, tw, bias, T, d, N, idx, gates, s);
-    case 6: return launch_router_tc_k<BN, STAGES, 6>(tx, tw, bias, T, d, N, idx, gates, s);
-    case 7: return launch_router_tc_k<BN, STAGES, 7>(tx, tw, bias, T, d, N, idx, gates, s);
-    default: return launch_router_tc_k<BN, STAGES, 8>(tx, tw, bias, T, d, N, idx, gates, s);
+    case 1: return launch_router_tc_k<BN, STAGES, 1>(tx, tw, bias, T, d, N, idx, gates, cc, s);
+    case 2: return launch_router_tc_k<BN, STAGES, 2>(tx, tw, bias, T, d, N, idx, gates, cc, s);
+    case 3: return launch_router_tc_k<BN, STAGES, 3>(tx, tw, bias, T, d, N, idx, gates, cc, s);
+    case 4: return launch_router_tc_k<BN, STAGES, 4>(tx, tw, bias, T, d, N, idx, gates, cc, s);
+    case 5: return launch_router_tc_k<BN, STAGES, 5>(tx, tw, bias, T, d, N, idx, gates, cc, s);
+    case 6: return launch_router_tc_k<BN, STAGES, 6>(tx, tw, bias, T, d, N, idx, gates, cc, s);
+    case 7: return launch_router_tc_k<BN, STAGES, 7>(tx, tw, bias, T, d, N, idx, gates, cc, s);
+    default: return launch_router_tc_k<BN, STAGES, 8>(tx, tw, bias, T, d, N, idx, gates, cc, s);
   }
 }
 
@@ -462,14 +465,17 @@ int forward_body(const bfmoe_layer* layer, const void* x, bool bf16, int T, int 
   if (e != cudaSuccess) return cuda_fail(e, "forward: pre-rotation");
 
   if (bf16 && d >= 64) {
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tbh;
     const int BN = std::min(d, 256);
-    if (!make_tmap_bf16(&ta, xrot, d, R, kGemmBM) || !make_tmap_bf16(&tb, wbf, d, d, BN))
+    if (!make_tmap_bf16(&ta, xrot, d, R, kGemmBM) || !make_tmap_bf16(&tb, wbf, d, d, BN) ||
+        !make_tmap_bf16(&tbh, wbf, d, d, BN >= 128 ? BN / 2 : BN))
       return fail(BFMOE_ECUDA, "forward: tensor map encoding failed");
+    __nv_bfloat16* zb = static_cast<__nv_bfloat16*>(z);
+    const int Ri = static_cast<int>(R);
     switch (BN) {
-      case 64: e = launch_gemm_tc<64, 8>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
-      case 128: e = launch_gemm_tc<128, 6>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
-      default: e = launch_gemm_tc<256, 4>(ta, tb, static_cast<__nv_bfloat16*>(z), static_cast<int>(R), d, layer->alpha, s); break;
+      case 64: e = launch_gemm_tc<64, 8>(ta, tb, tbh, zb, Ri, d, layer->alpha, s); break;
+      case 128: e = launch_gemm_tc<128, 6>(ta, tb, tbh, zb, Ri, d, layer->alpha, s); break;
+      default: e = launch_gemm_tc<256, 4>(ta, tb, tbh, zb, Ri, d, layer->alpha, s); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "forward: tensor-core GEMM");
   } else {
@@ -639,7 +645,8 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
   int32_t* totals = reinterpret_cast<int32_t*>(W + p.totals);
   const long long R = static_cast<long long>(T) * k;
 
-  if (x_dtype == BFMOE_BF16 && d % kGemmBK == 0) {
+  const bool tc_router = x_dtype == BFMOE_BF16 && d % kGemmBK == 0;
+  if (tc_router) {
     // tensor cores: exact 3-way bf16 split of W_g, top-k fused in the epilogue
     if (!aligned16(x)) return fail(BFMOE_EINVAL, "router_topk: x must be 16-byte aligned");
     __nv_bfloat16* parts = reinterpret_cast<__nv_bfloat16*>(W + p.wg_parts);
@@ -651,10 +658,10 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
     if (!make_tmap_bf16(&tx, x, d, T, kGemmBM) || !make_tmap_bf16(&tw, parts, d, 3LL * N, BN))
       return fail(BFMOE_ECUDA, "router_topk: tensor map encoding failed");
     switch (BN) {
-      case 16: e = launch_router_tc<16, 4>(tx, tw, bias, T, d, N, k, idx, gates, s); break;
-      case 32: e = launch_router_tc<32, 4>(tx, tw, bias, T, d, N, k, idx, gates, s); break;
-      case 64: e = launch_router_tc<64, 4>(tx, tw, bias, T, d, N, k, idx, gates, s); break;
-      default: e = launch_router_tc<128, 3>(tx, tw, bias, T, d, N, k, idx, gates, s); break;
+      case 16: e = launch_router_tc<16, 4>(tx, tw, bias, T, d, N, k, idx, gates, cc, s); break;
+      case 32: e = launch_router_tc<32, 4>(tx, tw, bias, T, d, N, k, idx, gates, cc, s); break;
+      case 64: e = launch_router_tc<64, 4>(tx, tw, bias, T, d, N, k, idx, gates, cc, s); break;
+      default: e = launch_router_tc<128, 3>(tx, tw, bias, T, d, N, k, idx, gates, cc, s); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "router_topk: tensor-core router");
   } else {
@@ -674,7 +681,8 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
     if (e != cudaSuccess) return cuda_fail(e, "router_topk: top-k");
   }
 
-  const int nchunks = static_cast<int>((R + kBucketChunk - 1) / kBucketChunk);
+  const int chunk = bucket_chunk(k);
+  const int nchunks = static_cast<int>((R + chunk - 1) / chunk);
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(bucket_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BFMOE_MAX_EXPERTS * 4);
@@ -682,13 +690,15 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
                          BFMOE_MAX_EXPERTS * 36 + 16);
     attr = true;
   }
-  e = launch("bucket_count", s, [&] { bucket_count_kernel<<<nchunks, 1024, N * 4, s>>>(idx, R, N, cc); });
-  if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket count");
+  if (!tc_router) {  // the tensor-core router writes the chunk histograms itself
+    e = launch("bucket_count", s, [&] { bucket_count_kernel<<<nchunks, chunk, N * 4, s>>>(idx, R, N, cc); });
+    if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket count");
+  }
   e = launch("bucket_scan", s, [&] { bucket_scan_kernel<<<(N + 31) / 32, 1024, 0, s>>>(cc, nchunks, N, totals); });
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scan");
   const size_t scatter_smem = ((N + 1) * 4 + 15) / 16 * 16 + static_cast<size_t>(N) * 32;
   e = launch("bucket_scatter", s, [&] {
-    bucket_scatter_kernel<<<nchunks, 1024, scatter_smem, s>>>(idx, R, N, cc, totals, counts, offsets, rows);
+    bucket_scatter_kernel<<<nchunks, chunk, scatter_smem, s>>>(idx, R, N, cc, totals, counts, offsets, rows);
   });
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scatter");
   return ok();

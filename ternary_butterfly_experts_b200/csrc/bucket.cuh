@@ -2,8 +2,10 @@
 // r = t*k + j by expert.  Within an expert, rows come in ascending r, which is
 // ascending token order because a token's k experts are distinct.
 //
-// Rows are cut into chunks of kBucketChunk (one 1024-thread block each):
-//   count    per-chunk expert histogram
+// Rows are cut into chunks of 128*k rows, the routed rows of 128 tokens (one
+// block of 128*k threads each):
+//   count    per-chunk expert histogram (the tensor-core router writes it from
+//            its epilogue; this kernel serves the float32 router)
 //   scan     per expert, exclusive prefix over chunks (+ totals)
 //   scatter  offsets = exclusive prefix over experts (each block); position =
 //            offsets[e] + chunk prefix + earlier warps of the chunk + rank
@@ -13,14 +15,15 @@
 
 namespace bfmoe {
 
-constexpr int kBucketChunk = 1024;
+// Routed rows per bucket chunk: those of 128 tokens (k <= 8, so <= 1024).
+__host__ __device__ constexpr int bucket_chunk(int k) { return 128 * k; }
 
 __global__ __launch_bounds__(1024) void bucket_count_kernel(const int32_t* __restrict__ idx, long long R, int N,
                                                             int32_t* __restrict__ chunk_counts) {
   extern __shared__ int cnt[];
   for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
-  const long long r = static_cast<long long>(blockIdx.x) * kBucketChunk + threadIdx.x;
+  const long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (r < R) {
     const int e = idx[r];
     if (e >= 0 && e < N) {
@@ -69,17 +72,16 @@ __global__ __launch_bounds__(1024) void bucket_scan_kernel(int32_t* __restrict__
 }
 
 // Exclusive prefix sum of totals[0..N) into off[0..N] (shared memory), by a
-// block of 1024 threads, N <= 4096 (4 experts per thread).
+// block of any multiple of 32 threads up to 1024; thread i sums experts
+// i*per .. i*per + per - 1.
 __device__ __forceinline__ void block_exclusive_scan(const int32_t* __restrict__ totals, int N, int* off) {
   __shared__ int warp_sum[32];
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  int v[4];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  const int per = (N + blockDim.x - 1) / blockDim.x;
   int local = 0;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int e = tid * 4 + q;
-    v[q] = e < N ? totals[e] : 0;
-    local += v[q];
+  for (int q = 0; q < per; ++q) {
+    const int e = tid * per + q;
+    local += e < N ? totals[e] : 0;
   }
   int incl = local;
 #pragma unroll
@@ -90,7 +92,7 @@ __device__ __forceinline__ void block_exclusive_scan(const int32_t* __restrict__
   if (lane == 31) warp_sum[w] = incl;
   __syncthreads();
   if (w == 0) {
-    const int ws = warp_sum[lane];
+    const int ws = lane < nw ? warp_sum[lane] : 0;
     int inc = ws;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -101,13 +103,14 @@ __device__ __forceinline__ void block_exclusive_scan(const int32_t* __restrict__
   }
   __syncthreads();
   int run = warp_sum[w] + incl - local;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int e = tid * 4 + q;
-    if (e < N) off[e] = run;
-    run += v[q];
+  for (int q = 0; q < per; ++q) {
+    const int e = tid * per + q;
+    if (e < N) {
+      off[e] = run;
+      run += totals[e];
+    }
   }
-  if (tid == 1023) off[N] = run;
+  if (tid == static_cast<int>(blockDim.x) - 1) off[N] = run;
   __syncthreads();
 }
 
@@ -132,7 +135,7 @@ __global__ __launch_bounds__(1024) void bucket_scatter_kernel(const int32_t* __r
       if (e < N) counts_out[e] = totals[e];
     }
   }
-  const long long r = static_cast<long long>(blockIdx.x) * kBucketChunk + tid;
+  const long long r = static_cast<long long>(blockIdx.x) * blockDim.x + tid;
   int e = -1 - lane;
   bool valid = false;
   if (r < R) {

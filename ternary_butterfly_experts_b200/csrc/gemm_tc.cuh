@@ -5,7 +5,12 @@
 // expert, all R routed rows form one dense GEMM; no grouped GEMM is needed.
 // The ternary weights are exact in bf16; the product accumulates in fp32.
 //
-// Persistent kernel, one CTA per SM, 128 x BN output tiles:
+// Persistent kernel, one CTA per SM, 128 x BN output tiles.  The tiles that
+// would form a last, partial wave are cut into 128 x BN/2 halves, so that no
+// CTA runs a whole tile more than the others; each tile walks its k-blocks
+// from a different start, so that the CTAs do not read the same B tile from
+// L2 at the same moment (each output is still one float32 sum of exact
+// products, in an order fixed per tile).
 //   warp 0 (one lane)  TMA producer: 128x64 A and BNx64 B tiles (128-byte
 //                      swizzle) into a STAGES-deep shared-memory ring;
 //   warp 1 (one lane)  MMA issuer: tcgen05.mma M=128 N=BN K=16 into one of two
@@ -34,9 +39,41 @@ struct GemmTcCfg {
   static constexpr uint32_t TMEM_COLS = 2 * BN;
 };
 
+// Work item i of the kernel: a whole tile, or a half of one of the last
+// tiles.
+struct GemmItem {
+  int m0, n0, n;  // rows m0.., columns n0 .. n0+n-1
+  int rot;        // first k-block
+};
+template <int BN>
+__device__ __forceinline__ GemmItem gemm_item(int i, int n_full, int n_tiles_n, int nk) {
+  int t, half = -1;
+  if (i < n_full) {
+    t = i;
+  } else {
+    t = n_full + (i - n_full) / 2;
+    half = (i - n_full) & 1;
+  }
+  GemmItem it;
+  it.m0 = (t / n_tiles_n) * kGemmBM;
+  it.n0 = (t % n_tiles_n) * BN + (half > 0 ? BN / 2 : 0);
+  it.n = half >= 0 ? BN / 2 : BN;
+  it.rot = t % nk;
+  return it;
+}
+
+// Items: whole tiles up to the last full wave of the grid, then the rest in
+// halves (when BN/2 is a valid MMA width).
+__host__ __device__ inline void gemm_items(int n_tiles, int grid, int bn, int* n_full, int* n_items) {
+  const int full = (bn >= 128) ? (n_tiles / grid) * grid : n_tiles;
+  *n_full = full;
+  *n_items = full + 2 * (n_tiles - full);
+}
+
 template <int BN, int STAGES>
 __global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                                                                           const __grid_constant__ CUtensorMap tmB,
+                                                                          const __grid_constant__ CUtensorMap tmBh,
                                                                           __nv_bfloat16* __restrict__ Z, int R, int d,
                                                                           float alpha) {
   using Cfg = GemmTcCfg<BN, STAGES>;
@@ -54,6 +91,8 @@ __global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const 
   const int nk = d / kGemmBK;
   const int n_tiles_n = d / BN;
   const int n_tiles = ((R + kGemmBM - 1) / kGemmBM) * n_tiles_n;
+  int n_full, n_items;
+  gemm_items(n_tiles, gridDim.x, BN, &n_full, &n_items);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -67,6 +106,7 @@ __global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const 
     mbar_fence_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmBh);
   }
   if (warp == 0) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
   tc_fence_before();
@@ -77,30 +117,34 @@ __global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const 
   if (warp == 0) {
     if (lane == 0) {
       int it = 0;
-      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-        const int m0 = (t / n_tiles_n) * kGemmBM, n0 = (t % n_tiles_n) * BN;
+      for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
+        const GemmItem w = gemm_item<BN>(i, n_full, n_tiles_n, nk);
         bool alive = true;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int ki = 0; ki < nk; ++ki, ++it) {
+          const int kb = (ki + w.rot) % nk;
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (it >= STAGES && !mbar_wait(empty + s, ph ^ 1u, 0x100u | s)) {
             alive = false;
             break;
           }
-          mbar_expect_tx(full + s, Cfg::STAGE_BYTES);
+          const bool half = w.n < BN;
+          mbar_expect_tx(full + s, Cfg::A_BYTES + (half ? Cfg::B_BYTES / 2 : Cfg::B_BYTES));
           uint8_t* a = smem + s * Cfg::STAGE_BYTES;
-          tma_load_2d(a, &tmA, full + s, kb * kGemmBK, m0);
-          tma_load_2d(a + Cfg::A_BYTES, &tmB, full + s, kb * kGemmBK, n0);
+          tma_load_2d(a, &tmA, full + s, kb * kGemmBK, w.m0);
+          tma_load_2d(a + Cfg::A_BYTES, half ? &tmBh : &tmB, full + s, kb * kGemmBK, w.n0);
         }
         if (!alive) break;
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, BN);
+      constexpr uint32_t idesc_full = idesc_bf16_f32(kGemmBM, BN);
+      constexpr uint32_t idesc_half = idesc_bf16_f32(kGemmBM, BN >= 128 ? BN / 2 : BN);
       int it = 0, i = 0;
       bool alive = true;
-      for (int t = blockIdx.x; t < n_tiles && alive; t += gridDim.x, ++i) {
+      for (int wi = blockIdx.x; wi < n_items && alive; wi += gridDim.x, ++i) {
+        const uint32_t idesc = wi < n_full ? idesc_full : idesc_half;
         const int buf = i & 1;
         if (i >= 2 && !mbar_wait(tempty + buf, ((i >> 1) - 1) & 1u, 0x300u | buf)) break;
         tc_fence_after();
@@ -129,19 +173,20 @@ __global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const 
     const int sp = warp & 3;
     uint32_t* buf_w = epi + (warp - 2) * 32 * 16;  // 32 rows x 16 bf16 pairs
     int i = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
-      const int m0 = (t / n_tiles_n) * kGemmBM, n0 = (t % n_tiles_n) * BN;
+    for (int wi = blockIdx.x; wi < n_items; wi += gridDim.x, ++i) {
+      const GemmItem w = gemm_item<BN>(wi, n_full, n_tiles_n, nk);
+      const int m0 = w.m0, n0 = w.n0;
       const int buf = i & 1;
       if (!mbar_wait(tfull + buf, (i >> 1) & 1u, 0x400u | buf)) break;
       tc_fence_after();
       const uint32_t base = tmem + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(buf * BN);
       const int row0 = m0 + sp * 32;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = 0; c < w.n; c += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(base + static_cast<uint32_t>(c), v);
         tmem_wait_ld();
-        if (c + 32 >= BN) {
+        if (c + 32 >= w.n) {
           // whole accumulator read: hand it back to the MMA warp
           tc_fence_before();
           __syncwarp();

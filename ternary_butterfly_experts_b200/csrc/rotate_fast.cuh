@@ -395,21 +395,26 @@ __device__ __forceinline__ void to_layout1(float (&r)[E], float* buf, int lane) 
   __syncwarp();
 }
 
-// ---- kernels: each warp stages its own rows in shared memory --------------------
+// ---- kernels: persistent warps, rows double-buffered in shared memory ----------
 //
-// Warp w of CTA b takes G consecutive bucket positions.  Lanes 0..G-1 read
-// their rows' ids and experts; the warp copies its G gathered rows into its
-// own slice of shared memory with cp.async and waits only for its own copies,
-// so there is no CTA-wide barrier: one warp's load latency overlaps the
-// arithmetic of the others.  A group whose rows share one expert is rotated
-// together (G rows per cos/sin load, tables read through L1); a mixed group
-// row by row.
+// The bucket positions are cut into groups of G consecutive positions.  The
+// grid is sized to what stays resident; CTA b takes an even, contiguous range
+// of groups and its warp w takes groups w, w + WARPS, w + 2*WARPS, ... of that
+// range, so the warps of a CTA work on neighbouring positions (mostly one
+// expert, whose cos/sin table they share through L1).  A warp first reads the
+// ids, experts and gates of all its rows (lane l holds row l % G of its group
+// l / G), then walks its groups with two shared-memory row buffers: while it
+// rotates group j, cp.async brings in group j + 1.  A group whose rows share
+// one expert is rotated together (G rows per cos/sin load); a mixed or partial
+// group row by row.  No CTA-wide barrier is used.
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // 16-byte chunk c of a staged row sits at chunk c ^ ((c >> 3) & 7): layout-1
@@ -423,11 +428,36 @@ struct StagedCfg {
   static constexpr int THREADS = Gm::WARPS * 32;
   static constexpr size_t TAB_QUADS = tab_quads(E);
   static constexpr int MIN_BLOCKS = E <= 32 ? 2 : 1;
-  // per warp: its G staged rows and one float32 transpose buffer
-  static constexpr size_t WARP_BYTES = G * Gm::D * sizeof(Tin) + Gm::D * 4;
+  static constexpr int MAXJ = 32 / G;  // groups per warp (one row's metadata per lane)
+  // per warp: two buffers of G staged rows and one float32 transpose buffer
+  static constexpr size_t BUF_BYTES = G * Gm::D * sizeof(Tin);
+  static constexpr size_t WARP_BYTES = 2 * BUF_BYTES + Gm::D * 4;
   static constexpr size_t SMEM = Gm::WARPS * WARP_BYTES;
-  static constexpr int ROWS = Gm::WARPS * G;  // bucket positions per CTA
 };
+
+// Grid for `groups` groups when `resident` CTAs fit on the device at once.
+template <int E, typename Tin>
+__host__ inline int staged_grid(long long groups, int resident) {
+  using C = StagedCfg<E, Tin>;
+  const long long per = static_cast<long long>(C::Gm::WARPS);
+  long long g = (groups + per - 1) / per;                               // one group per warp at most
+  const long long need = (groups + per * C::MAXJ - 1) / (per * C::MAXJ);  // MAXJ groups per warp at least
+  const long long want = resident > need ? resident : need;
+  if (g > want) g = want;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+// The groups of warp w of this CTA: gb0 + w + WARPS*j for j < nj.
+struct WarpGroups {
+  long long gb0;
+  int nj;
+};
+template <int WARPS>
+__device__ __forceinline__ WarpGroups warp_groups(long long groups, int w) {
+  const long long gb0 = blockIdx.x * groups / gridDim.x, gb1 = (blockIdx.x + 1) * groups / gridDim.x;
+  const long long n = gb1 - gb0 - w;
+  return WarpGroups{gb0, n > 0 ? static_cast<int>((n + WARPS - 1) / WARPS) : 0};
+}
 
 struct RowMeta {
   int row;    // routed row r = t*k + j (or -1)
@@ -435,7 +465,7 @@ struct RowMeta {
   float gate;
 };
 
-// Lane g < G reads bucket position p0 + g: its row, expert and gate.
+// Row metadata of bucket position p: its row, expert and gate.
 __device__ __forceinline__ RowMeta fetch_row_meta(const int32_t* __restrict__ rows, const int32_t* __restrict__ idx,
                                                   const float* __restrict__ gates, long long p, long long R, int N) {
   RowMeta m{-1, -1, 0.f};
@@ -483,45 +513,72 @@ __global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS, StagedCfg<E, Tin>::MIN_
   constexpr int G = C::G, D = Gm::D;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const long long p0 = (static_cast<long long>(blockIdx.x) * Gm::WARPS + w) * G;
-  if (p0 >= R) return;
-  uint8_t* wbase = smem_raw + w * C::WARP_BYTES;
-  Tin* xs = reinterpret_cast<Tin*>(wbase);
-  float* buf = reinterpret_cast<float*>(wbase + G * D * sizeof(Tin));
-
-  const RowMeta mine = lane < G ? fetch_row_meta(rows, idx, nullptr, p0 + lane, R, N) : RowMeta{-1, -1, 0.f};
-  const int my_tok = mine.row >= 0 ? mine.row / k : 0;  // invalid rows read token 0; output zeroed
-  constexpr int CH = D * sizeof(Tin) / 16;
-  for (int i = lane; i < G * CH; i += 32) {
-    const int g = i / CH, c = i % CH;
-    const int t = __shfl_sync(__activemask(), my_tok, g);
-    cp_async16(reinterpret_cast<uint8_t*>(xs) + static_cast<size_t>(g) * D * sizeof(Tin) + c * 16,
-               reinterpret_cast<const uint8_t*>(x + static_cast<size_t>(t) * D) + c * 16);
-  }
-  cp_async_wait_all();
-  __syncwarp();
-
-  const int e0 = __shfl_sync(FULL_MASK, mine.ex, 0);
-  const unsigned same = __ballot_sync(FULL_MASK, lane < G && mine.ex >= 0 && mine.ex == e0);
-  if (same == (1u << G) - 1u && p0 + G <= R) {
-    pre_rotate_rows_smem<Gm, G, Tin, Tout>(xs, quads + static_cast<size_t>(e0) * C::TAB_QUADS, xrot + p0 * D, buf,
-                                           lane);
+  const long long groups = (R + G - 1) / G;
+  const WarpGroups wg = warp_groups<Gm::WARPS>(groups, w);
+  if (wg.nj == 0) return;
+  if (wg.nj > C::MAXJ) {  // the host sizes the grid so that this cannot happen
+    if (lane == 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(wg.nj));
     return;
   }
-#pragma unroll 1
-  for (int g = 0; g < G; ++g) {
-    const long long p = p0 + g;
-    if (p >= R) break;
-    const int e = __shfl_sync(FULL_MASK, mine.ex, g);
-    if (e < 0) {
-      float z[E];
-#pragma unroll
-      for (int q = 0; q < E; ++q) z[q] = 0.f;
-      store_row<E, Tout>(xrot + p * D + lane * E, z, true);
-      continue;
+  uint8_t* wbase = smem_raw + w * C::WARP_BYTES;
+  Tin* xs = reinterpret_cast<Tin*>(wbase);
+  float* buf = reinterpret_cast<float*>(wbase + 2 * C::BUF_BYTES);
+  auto pos0 = [&](int j) { return (wg.gb0 + w + static_cast<long long>(Gm::WARPS) * j) * G; };
+
+  const int jl = lane / G;
+  const RowMeta mine = jl < wg.nj ? fetch_row_meta(rows, idx, nullptr, pos0(jl) + lane % G, R, N)
+                                  : RowMeta{-1, -1, 0.f};
+  const int my_tok = mine.row >= 0 ? mine.row / k : 0;  // invalid rows read token 0; output zeroed
+
+  constexpr int CH = D * sizeof(Tin) / 16;  // 16-byte chunks per row; G*CH is a multiple of 32
+  auto issue = [&](int j) {
+    uint8_t* dst = reinterpret_cast<uint8_t*>(xs) + (j & 1) * C::BUF_BYTES;
+#pragma unroll 4
+    for (int i = lane; i < G * CH; i += 32) {
+      const int g = i / CH, c = i % CH;
+      const int t = __shfl_sync(FULL_MASK, my_tok, j * G + g);
+      cp_async16(dst + static_cast<size_t>(g) * D * sizeof(Tin) + c * 16,
+                 reinterpret_cast<const uint8_t*>(x + static_cast<size_t>(t) * D) + c * 16);
     }
-    pre_rotate_rows_smem<Gm, 1, Tin, Tout>(xs + g * D, quads + static_cast<size_t>(e) * C::TAB_QUADS, xrot + p * D,
-                                           buf, lane);
+    cp_async_commit();
+  };
+
+  issue(0);
+#pragma unroll 1
+  for (int j = 0; j < wg.nj; ++j) {
+    if (j + 1 < wg.nj) {
+      issue(j + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+    const Tin* cur = xs + (j & 1) * G * D;
+    const long long p0 = pos0(j);
+    const int e0 = __shfl_sync(FULL_MASK, mine.ex, j * G);
+    const unsigned gm = ((1u << G) - 1u) << (j * G);
+    const unsigned same = __ballot_sync(FULL_MASK, mine.ex >= 0 && mine.ex == e0) & gm;
+    if (same == gm && p0 + G <= R) {
+      pre_rotate_rows_smem<Gm, G, Tin, Tout>(cur, quads + static_cast<size_t>(e0) * C::TAB_QUADS, xrot + p0 * D,
+                                             buf, lane);
+    } else {
+#pragma unroll 1
+      for (int g = 0; g < G; ++g) {
+        const long long p = p0 + g;
+        if (p >= R) break;
+        const int e = __shfl_sync(FULL_MASK, mine.ex, j * G + g);
+        if (e < 0) {
+          float z[E];
+#pragma unroll
+          for (int q = 0; q < E; ++q) z[q] = 0.f;
+          store_row<E, Tout>(xrot + p * D + lane * E, z, true);
+          continue;
+        }
+        pre_rotate_rows_smem<Gm, 1, Tin, Tout>(cur + g * D, quads + static_cast<size_t>(e) * C::TAB_QUADS,
+                                               xrot + p * D, buf, lane);
+      }
+    }
+    __syncwarp();  // buffer j & 1 is refilled by issue(j + 2)
   }
 }
 
@@ -574,39 +631,67 @@ __global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS, StagedCfg<E, Tz>::MIN_BL
   constexpr int G = C::G, D = Gm::D;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const long long p0 = (static_cast<long long>(blockIdx.x) * Gm::WARPS + w) * G;
-  if (p0 >= R) return;
-  uint8_t* wbase = smem_raw + w * C::WARP_BYTES;
-  Tz* zs = reinterpret_cast<Tz*>(wbase);
-  float* buf = reinterpret_cast<float*>(wbase + G * D * sizeof(Tz));
-
-  const RowMeta mine = lane < G ? fetch_row_meta(rows, idx, gates, p0 + lane, R, N) : RowMeta{-1, -1, 0.f};
-  constexpr int CH = D * sizeof(Tz) / 16;  // 16-byte chunks per row
-  for (int i = lane; i < G * CH; i += 32) {
-    const int g = i / CH, c = i % CH;
-    const long long p = p0 + g < R ? p0 + g : R - 1;
-    cp_async16(reinterpret_cast<uint8_t*>(zs) + static_cast<size_t>(g) * D * sizeof(Tz) + 16 * chunk_swz(c),
-               reinterpret_cast<const uint8_t*>(z + p * D) + 16 * c);
-  }
-  cp_async_wait_all();
-  __syncwarp();
-
-  const int e0 = __shfl_sync(FULL_MASK, mine.ex, 0);
-  const unsigned same = __ballot_sync(FULL_MASK, lane < G && mine.ex >= 0 && mine.ex == e0);
-  if (same == (1u << G) - 1u && p0 + G <= R) {
-    RowMeta m[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, g);
-    post_rotate_rows_smem<Gm, G, Tz, Ts>(zs, quads + static_cast<size_t>(e0) * C::TAB_QUADS, m, slot, buf, lane);
+  const long long groups = (R + G - 1) / G;
+  const WarpGroups wg = warp_groups<Gm::WARPS>(groups, w);
+  if (wg.nj == 0) return;
+  if (wg.nj > C::MAXJ) {  // the host sizes the grid so that this cannot happen
+    if (lane == 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(wg.nj));
     return;
   }
+  uint8_t* wbase = smem_raw + w * C::WARP_BYTES;
+  Tz* zs = reinterpret_cast<Tz*>(wbase);
+  float* buf = reinterpret_cast<float*>(wbase + 2 * C::BUF_BYTES);
+  auto pos0 = [&](int j) { return (wg.gb0 + w + static_cast<long long>(Gm::WARPS) * j) * G; };
+
+  const int jl = lane / G;
+  const RowMeta mine = jl < wg.nj ? fetch_row_meta(rows, idx, gates, pos0(jl) + lane % G, R, N)
+                                  : RowMeta{-1, -1, 0.f};
+
+  constexpr int CH = D * sizeof(Tz) / 16;  // 16-byte chunks per row; G*CH is a multiple of 32
+  auto issue = [&](int j) {
+    uint8_t* dst = reinterpret_cast<uint8_t*>(zs) + (j & 1) * C::BUF_BYTES;
+    const long long p0 = pos0(j);
+#pragma unroll 4
+    for (int i = lane; i < G * CH; i += 32) {
+      const int g = i / CH, c = i % CH;
+      const long long p = p0 + g < R ? p0 + g : R - 1;
+      cp_async16(dst + static_cast<size_t>(g) * D * sizeof(Tz) + 16 * chunk_swz(c),
+                 reinterpret_cast<const uint8_t*>(z + p * D) + 16 * c);
+    }
+    cp_async_commit();
+  };
+
+  issue(0);
 #pragma unroll 1
-  for (int g = 0; g < G; ++g) {
-    if (p0 + g >= R) break;
-    const RowMeta m1[1] = {shfl_meta(mine, g)};
-    if (m1[0].ex < 0) continue;
-    post_rotate_rows_smem<Gm, 1, Tz, Ts>(zs + g * D, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS, m1, slot,
-                                         buf, lane);
+  for (int j = 0; j < wg.nj; ++j) {
+    if (j + 1 < wg.nj) {
+      issue(j + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+    const Tz* cur = zs + (j & 1) * G * D;
+    const long long p0 = pos0(j);
+    const int e0 = __shfl_sync(FULL_MASK, mine.ex, j * G);
+    const unsigned gm = ((1u << G) - 1u) << (j * G);
+    const unsigned same = __ballot_sync(FULL_MASK, mine.ex >= 0 && mine.ex == e0) & gm;
+    if (same == gm && p0 + G <= R) {
+      RowMeta m[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, j * G + g);
+      post_rotate_rows_smem<Gm, G, Tz, Ts>(cur, quads + static_cast<size_t>(e0) * C::TAB_QUADS, m, slot, buf, lane);
+    } else {
+#pragma unroll 1
+      for (int g = 0; g < G; ++g) {
+        if (p0 + g >= R) break;
+        const RowMeta m1[1] = {shfl_meta(mine, j * G + g)};
+        if (m1[0].ex < 0) continue;
+        post_rotate_rows_smem<Gm, 1, Tz, Ts>(cur + g * D, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS, m1,
+                                             slot, buf, lane);
+      }
+    }
+    __syncwarp();  // buffer j & 1 is refilled by issue(j + 2)
   }
 }
 

@@ -15,7 +15,9 @@
 // chunk's columns), each keeping a running top-k of its half (larger logit
 // first, lower expert index on ties, NaN below every number) while the next
 // chunk is being multiplied; the two partial lists of a row are merged through
-// shared memory, and the row's idx and renormalised gates are written.
+// shared memory, and the row's idx and renormalised gates are written.  The
+// CTA's 128*k routed rows form one bucket chunk: the epilogue also writes
+// their expert histogram (chunk_counts[blockIdx.x][e]).
 #pragma once
 #include "common.cuh"
 #include "gemm_tc.cuh"
@@ -88,7 +90,8 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
                                                            const __grid_constant__ CUtensorMap tmW,
                                                            const float* __restrict__ bias, int T, int d, int N,
                                                            int32_t* __restrict__ idx,
-                                                           float* __restrict__ gates) {
+                                                           float* __restrict__ gates,
+                                                           int32_t* __restrict__ chunk_counts) {
   using Cfg = RouterTcCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -105,6 +108,11 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
   const int m0 = blockIdx.x * kGemmBM;
   const int nk = d / kGemmBK;
   const int nchunks = (N + BN - 1) / BN;
+  // CTAs start at different k-blocks and expert chunks, so that they do not
+  // all read the same weight tile from L2 at the same moment.  Each logit is
+  // still one float32 sum of exact products, in an order fixed per CTA.
+  const int k_rot = blockIdx.x % nk;
+  const int c_rot = (blockIdx.x / nk) % nchunks;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -129,8 +137,10 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
   if (warp == 0 && lane == 0) {
     int it = 0;
     bool alive = true;
-    for (int c = 0; c < nchunks && alive; ++c) {
-      for (int kb = 0; kb < nk; ++kb, ++it) {
+    for (int ci = 0; ci < nchunks && alive; ++ci) {
+      const int c = (ci + c_rot) % nchunks;
+      for (int ki = 0; ki < nk; ++ki, ++it) {
+        const int kb = (ki + k_rot) % nk;
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
         if (it >= STAGES && !mbar_wait(empty + s, ph ^ 1u, 0x1100u | s)) {
@@ -154,7 +164,7 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
       if (c >= 2 && !mbar_wait(acc_empty + buf, ((c >> 1) - 1) & 1u, 0x1300u | buf)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * BN);
-      for (int kb = 0; kb < nk; ++kb, ++it) {
+      for (int kb = 0; kb < nk; ++kb, ++it) {  // kb counts k-blocks in arrival order
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
         if (!mbar_wait(full + s, ph, 0x1200u | s)) {
@@ -193,9 +203,10 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
   TopK<K> top;
   top.init();
   bool ok = true;
-  for (int c = 0; c < nchunks; ++c) {
-    const int buf = c & 1;
-    if (!mbar_wait(acc_full + buf, (c >> 1) & 1u, 0x1400u | buf)) {
+  for (int ci = 0; ci < nchunks; ++ci) {
+    const int c = (ci + c_rot) % nchunks;
+    const int buf = ci & 1;
+    if (!mbar_wait(acc_full + buf, (ci >> 1) & 1u, 0x1400u | buf)) {
       ok = false;
       break;
     }
@@ -230,6 +241,11 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
     }
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kRouterEpiWarps * 32) : "memory");
+  // the bias is no longer read: its shared memory becomes the histogram
+  int* hist = reinterpret_cast<int*>(bias_s);
+  const int et = threadIdx.x - 64;  // 0 .. 255
+  for (int e = et; e < N; e += kRouterEpiWarps * 32) hist[e] = 0;
+  asm volatile("bar.sync 1, %0;" ::"r"(kRouterEpiWarps * 32) : "memory");
   if (hf == 0 && ok && row < T) {
 #pragma unroll
     for (int j = 0; j < K; ++j) top.push(merge_v[lr * BFMOE_MAX_K + j], merge_i[lr * BFMOE_MAX_K + j]);
@@ -245,8 +261,12 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
     for (int j = 0; j < K; ++j) {
       idx[static_cast<size_t>(row) * K + j] = top.id[j];
       gates[static_cast<size_t>(row) * K + j] = z[j] / sum;
+      if (top.id[j] < N) atomicAdd(&hist[top.id[j]], 1);
     }
   }
+  asm volatile("bar.sync 1, %0;" ::"r"(kRouterEpiWarps * 32) : "memory");
+  for (int e = et; e < N; e += kRouterEpiWarps * 32)
+    chunk_counts[static_cast<size_t>(blockIdx.x) * N + e] = hist[e];
   tc_fence_before();
   __syncthreads();
 }
