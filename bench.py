@@ -337,19 +337,24 @@ def run_ours(args, wl):
     B.bfmoe_profile_enable(False)
 
     # --- end to end through host buffers ----------------------------------------
-    # copy in from pinned host memory, the captured router + forward, copy out
+    # bfmoe_moe_forward_host: pinned host tokens in, pinned host outputs out,
+    # the copies overlapped with the work in token chunks; the call is
+    # captured once as a CUDA graph (copies included) and replayed per step
     x_host = inp.x.pin_memory()
     y_host = torch.empty(x.shape, dtype=x.dtype).pin_memory()
-
-    def e2e_step():
-        x.copy_(x_host, non_blocking=True)
-        graph.replay()
-        y_host.copy_(y, non_blocking=True)
+    model.forward_host(x_host, y_host)  # creates the copy streams before capture
+    torch.cuda.synchronize()
+    host_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(host_graph):
+        model.forward_host(x_host, y_host)
 
     for _ in range(2):
-        e2e_step()
-    e2e_ms = timed(args.steps, e2e_step)
+        host_graph.replay()
+    e2e_ms = timed(args.steps, host_graph.replay)
     e2e_ms = max_over_ranks(e2e_ms)
+    e2e_eager_ms = timed(args.steps, lambda: model.forward_host(x_host, y_host))
+    e2e_eager_ms = max_over_ranks(e2e_eager_ms)
+    B.bfmoe_check_device_error()
 
     if rank == 0:
         clk = clocks.summary()
@@ -363,7 +368,7 @@ def run_ours(args, wl):
                      "avg_us": 1e3 * ms / n}
             kernels[name] = entry
         dom = max(kt.items(), key=lambda kv: kv[1][1])[0]
-        roof = roofline_entry(dom, kt[dom], costs, peaks, clk)
+        roof = roofline_entry(dom, kt[dom], costs, peaks, clk, workload=wl.name)
         flops = 2.0 * T * wl.k * wl.d ** 2
         bytes_alg = algorithmic_bytes(wl)
         t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_alg / (peaks["hbm_gbs"] * 1e9))
@@ -385,14 +390,17 @@ def run_ours(args, wl):
             "cpu_baseline": None,
             "e2e": {"value": T * world * args.steps / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
-                    "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
+                    "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
+                    "call": "bfmoe_moe_forward_host (pinned host buffers, copies overlapped in token chunks), "
+                            "captured once as a CUDA graph and replayed per step",
+                    "eager_value": T * world * args.steps / (e2e_eager_ms / 1e3)},
             "gpu_launches": int(launches),
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(inp, args.cpu_fraction)
         print(json.dumps(line), flush=True)
-    del graph
+    del graph, host_graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -408,7 +416,52 @@ def algorithmic_bytes(wl):
             + T * k * 8)
 
 
-def roofline_entry(name, kt_entry, costs, peaks, clk):
+# Launch names of the library -> kernel names in the ncu summaries.
+NCU_KERNEL = {"post_rotate": "post_rotate_fast_kernel", "pre_rotate": "pre_rotate_fast_kernel",
+              "ternary_gemm_tc": "ternary_gemm_tc_kernel", "router_tc": "router_tc_kernel",
+              "combine": "combine_kernel", "rot_table": "rot_quads_kernel"}
+
+
+def kernel_sources_hash() -> str:
+    """sha256 over the library's CUDA sources (sorted by name)."""
+    import hashlib
+    d = os.path.join(ROOT, "ternary_butterfly_experts_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            with open(os.path.join(d, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(name, workload):
+    """DRAM bytes (read + write) of one launch of kernel `name` from the
+    committed ncu summary of this workload, or None when there is none or the
+    kernel sources have changed since it was taken."""
+    import glob
+    import re
+    kname = NCU_KERNEL.get(name)
+    if kname is None:
+        return None
+    src_hash = kernel_sources_hash()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"ncu_full_*_{workload}.md"))):
+        with open(path) as f:
+            text = f.read()
+        m = re.search(r"kernel sources sha256: ([0-9a-f]{64})", text)
+        if not m or m.group(1) != src_hash:
+            continue
+        sec = re.search(r"## `" + re.escape(kname) + r"[^`]*`(.*?)(?=\n## |\Z)", text, re.S)
+        if not sec:
+            continue
+        rd = re.search(r"dram__bytes_read\.sum \| ([0-9.]+) Mbyte", sec.group(1))
+        wr = re.search(r"dram__bytes_write\.sum \| ([0-9.]+) Mbyte", sec.group(1))
+        if rd and wr:
+            return (float(rd.group(1)) + float(wr.group(1))) * 1e6
+    return None
+
+
+def roofline_entry(name, kt_entry, costs, peaks, clk, workload=None):
     n, ms = kt_entry
     avg_s = ms / n / 1e3
     bound, work, unit = costs.get(name, ("hbm", float("nan"), "GB/s"))
@@ -425,9 +478,12 @@ def roofline_entry(name, kt_entry, costs, peaks, clk):
         achieved = work / avg_s / 1e9
         peak = peaks["hbm_gbs"]
         src = "hbm_gbs (measured copy)"
+    traffic = profiled_traffic(name, workload) if workload else None
     return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": None, "avg_launch_us": avg_s * 1e6,
-            "work_per_launch": work, "peak_source": src}
+            "frac": achieved / peak, "traffic": traffic, "avg_launch_us": avg_s * 1e6,
+            "work_per_launch": work, "peak_source": src,
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, first launch (profiles/)"
+            if traffic is not None else "no ncu summary taken from the current kernel sources"}
 
 
 def main():

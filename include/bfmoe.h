@@ -192,6 +192,41 @@ int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int 
 size_t bfmoe_moe_workspace_size(int d, int n_experts, int T, int k, int x_dtype);
 
 /*
+ * Router and expert forward from and to HOST memory, the host <-> device
+ * copies overlapped with the work.  The T tokens are cut into chunks of
+ * `chunk` tokens (chunk <= 0: about T/2, at least 2048; after a first chunk,
+ * the last chunk's worth is cut into halves down to 512 tokens, so that the
+ * unoverlapped work and copy of the last chunk are short); chunk i's copy in,
+ * chunk i-1's router + forward and chunk i-2's copy out run at the same time
+ * on a library-owned copy-in stream, `stream` and a library-owned copy-out
+ * stream, ordered with events.  Each token's output is that of
+ * bfmoe_moe_forward on its chunk (tokens are independent; the pages route
+ * every token on its own, summary 2.3).  The weight-only tables are built
+ * once per call.  Pages have no counterpart for the host interface.
+ *   x_host    host [T][d] (read), best page-locked: pageable memory makes the
+ *             copies synchronous
+ *   y_host    host [T][d] (written), same dtype; complete once the work
+ *             enqueued on `stream` by this call has finished (synchronise the
+ *             stream before reading it)
+ *   chunk     tokens per chunk, or <= 0 for the default
+ *   ws        device scratch of bfmoe_moe_host_workspace_size(...) bytes (the
+ *             device copies of x and y, one chunk's routing and one chunk's
+ *             bfmoe_moe_forward scratch), 256-byte aligned
+ * The copy streams and their events are created once per device on first use
+ * (make that first call before any stream capture); after that the whole call
+ * is stream-ordered and can be captured in a CUDA graph, copies included.
+ * Calls that overlap on one device share the copy streams and serialise there.
+ * Returns BFMOE_EINVAL for null pointers or bad sizes, BFMOE_EWORKSPACE for a
+ * short workspace.
+ */
+int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_dtype, int T,
+                           const float* w_gate, const float* bias, int k, void* y_host, int chunk,
+                           void* ws, size_t ws_bytes, bfmoe_stream_t stream);
+
+/* Scratch bytes that bfmoe_moe_forward_host needs (0 for invalid sizes). */
+size_t bfmoe_moe_host_workspace_size(int d, int n_experts, int T, int k, int x_dtype, int chunk);
+
+/*
  * Form expert e densely, alpha * B(phi_e) . W_base . B(theta_e)^T, in float32
  * (technical summary, 2.1).  For checking only.
  *   w_out     device float [d][d] (written), row = output

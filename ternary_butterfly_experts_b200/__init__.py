@@ -237,6 +237,33 @@ def bfmoe_moe_forward(layer: Layer, x, w_gate, bias, k: int, ws, routing=None, y
     return y, routing
 
 
+def bfmoe_moe_host_workspace_size(d: int, n_experts: int, T: int, k: int, x_dtype: int, chunk: int = 0) -> int:
+    return int(capi.lib().bfmoe_moe_host_workspace_size(d, n_experts, T, k, x_dtype, chunk))
+
+
+def bfmoe_moe_forward_host(layer: Layer, x_host, w_gate, bias, k: int, y_host, ws, chunk: int = 0, stream=None):
+    """Router + forward from and to host memory (pinned CPU tensors), the
+    copies overlapped with the work in chunks of ``chunk`` tokens.  ``y_host``
+    is complete once ``stream`` has been synchronised.  Returns y_host."""
+    torch = _torch()
+    for t, name in ((x_host, "x_host"), (y_host, "y_host")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    if y_host.shape != x_host.shape or y_host.dtype != x_host.dtype:
+        raise ValueError("y_host must match x_host in shape and dtype")
+    _need(w_gate, "w_gate", torch.float32)
+    if bias is not None:
+        _need(bias, "bias", torch.float32)
+    T, d = x_host.shape
+    if d != layer.d:
+        raise ValueError(f"x has width {d}, layer has d={layer.d}")
+    capi.check(capi.lib().bfmoe_moe_forward_host(
+        ctypes.byref(layer.c), ctypes.c_void_p(x_host.data_ptr()), _dtype_code(x_host), T, _ptr(w_gate), _ptr(bias),
+        k, ctypes.c_void_p(y_host.data_ptr()), chunk, _ptr(ws), ws.numel() if ws is not None else 0,
+        _stream(stream)))
+    return y_host
+
+
 def bfmoe_materialize_expert(layer: Layer, e: int, out=None, stream=None):
     """alpha * B(phi_e) . W_base . B(theta_e)^T as float32 [d][d] (checking aid)."""
     torch = _torch()
@@ -285,7 +312,6 @@ class ButterflyMoE:
         self.counts = torch.empty((N,), dtype=torch.int32, device=dev)
         self.offsets = torch.empty((N + 1,), dtype=torch.int32, device=dev)
         self.rows = torch.empty((max_tokens * k,), dtype=torch.int32, device=dev)
-        self.x_dev = torch.empty((max_tokens, d), dtype=x_dtype, device=dev)
         self.y_dev = torch.empty((max_tokens, d), dtype=x_dtype, device=dev)
 
     def route(self, x, stream=None):
@@ -305,11 +331,17 @@ class ButterflyMoE:
                                  stream=stream)
         return y
 
-    def forward_host(self, x_host, y_host, stream=None):
-        """Host -> device copy, router + forward, device -> host copy."""
+    def forward_host(self, x_host, y_host, chunk: int = 0, stream=None):
+        """The end-to-end call: pinned host tokens in, pinned host outputs back,
+        through bfmoe_moe_forward_host (copies overlapped with the work in
+        token chunks).  Synchronise ``stream`` before reading y_host."""
+        torch = _torch()
         T = x_host.shape[0]
-        xd = self.x_dev[:T]
-        xd.copy_(x_host, non_blocking=True)
-        y = self(xd, stream=stream)
-        y_host.copy_(y, non_blocking=True)
-        return y_host
+        key = (T, chunk)
+        if getattr(self, "_host_key", None) != key:
+            code = BFMOE_BF16 if self.dtype == torch.bfloat16 else BFMOE_F32
+            n = bfmoe_moe_host_workspace_size(self.layer.d, self.layer.n_experts, T, self.k, code, chunk)
+            self.ws_host = torch.empty(max(n, 256), dtype=torch.uint8, device=self.layer.theta.device)
+            self._host_key = key
+        return bfmoe_moe_forward_host(self.layer, x_host, self.w_gate, self.bias, self.k, y_host, self.ws_host,
+                                      chunk=chunk, stream=stream)

@@ -538,6 +538,90 @@ int side_stream(SideStream** out) {
   return BFMOE_OK;
 }
 
+// Copy streams and events of bfmoe_moe_forward_host, one set per device,
+// created on first use.
+constexpr int kHostMaxChunks = 64;
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t fork = nullptr, done = nullptr;
+  cudaEvent_t ev_in[kHostMaxChunks] = {}, ev_out[kHostMaxChunks] = {};
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[64];
+
+int host_pipe(HostPipe** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_forward_host: cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(BFMOE_EUNSUPPORTED, "moe_forward_host: device %d", dev);
+  std::lock_guard<std::mutex> lk(g_pipe_mu);
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.in) {
+    const unsigned ef = cudaEventDisableTiming;
+    if ((e = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&hp.fork, ef)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&hp.done, ef)) != cudaSuccess)
+      return cuda_fail(e, "moe_forward_host: copy streams");
+    for (int i = 0; i < kHostMaxChunks; ++i)
+      if ((e = cudaEventCreateWithFlags(&hp.ev_in[i], ef)) != cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&hp.ev_out[i], ef)) != cudaSuccess)
+        return cuda_fail(e, "moe_forward_host: events");
+  }
+  *out = &hp;
+  return BFMOE_OK;
+}
+
+// Workspace of bfmoe_moe_forward_host: device x and y, one chunk's routing,
+// one chunk's bfmoe_moe_forward scratch; and the chunk schedule.
+struct HostPlan {
+  int chunk, nchunks;
+  int start[kHostMaxChunks + 1];  // chunk c = tokens start[c] .. start[c+1]-1
+  size_t x_dev, y_dev, idx, gates, counts, offsets, rows, moe, total;
+};
+
+// Chunks of `chunk` tokens; after the first chunk, the last chunk's worth is
+// cut into halves (down to 512 tokens), so that the work and the copy out of
+// the last chunk, which nothing overlaps, are short.
+HostPlan make_host_plan(int d, int N, int T, int k, int xdt, int chunk) {
+  HostPlan h{};
+  if (chunk <= 0) chunk = std::max(2048, (T + 1) / 2);
+  chunk = (chunk + 127) / 128 * 128;
+  if (T > 0 && chunk > T) chunk = T;
+  if (T > 0 && (T + chunk - 1) / chunk > kHostMaxChunks / 2) chunk = (T + kHostMaxChunks / 2 - 1) / (kHostMaxChunks / 2);
+  h.chunk = std::max(1, chunk);
+  int t = 0, c = 0;
+  while (t < T) {
+    const int left = T - t;
+    int n = left > h.chunk ? h.chunk : left;
+    if (t > 0 && left <= h.chunk && n > 512) n = std::max(512, n / 2);  // taper the tail
+    if (c == kHostMaxChunks - 1) n = left;
+    h.start[c++] = t;
+    t += n;
+  }
+  h.start[c] = T;
+  h.nchunks = c;
+  const size_t es = xdt == BFMOE_BF16 ? 2 : 4;
+  const size_t rc = static_cast<size_t>(h.chunk) * k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  h.x_dev = take(static_cast<size_t>(T) * d * es);
+  h.y_dev = take(static_cast<size_t>(T) * d * es);
+  h.idx = take(rc * 4);
+  h.gates = take(rc * 4);
+  h.counts = take(static_cast<size_t>(N) * 4);
+  h.offsets = take(static_cast<size_t>(N + 1) * 4);
+  h.rows = take(rc * 4);
+  const Plan p = make_plan(d, N, h.chunk, k, xdt);
+  h.moe = take(p.fwd_end + p.rt_end);
+  h.total = off;
+  return h;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -733,6 +817,87 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
   uint8_t* W = static_cast<uint8_t*>(ws);
   if ((rc = build_weight_tables(layer, x_dtype == BFMOE_BF16, p, W, s))) return rc;
   return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, s);
+}
+
+size_t bfmoe_moe_host_workspace_size(int d, int n_experts, int T, int k, int x_dtype, int chunk) {
+  if (check_sizes(d, n_experts, T, k) != BFMOE_OK || check_dtype(x_dtype) != BFMOE_OK) return 0;
+  return make_host_plan(d, n_experts, T, k, x_dtype, chunk).total;
+}
+
+int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_dtype, int T, const float* w_gate,
+                           const float* bias, int k, void* y_host, int chunk, void* ws, size_t ws_bytes,
+                           bfmoe_stream_t stream) {
+  if (!layer) return fail(BFMOE_EINVAL, "moe_forward_host: NULL layer");
+  const int d = layer->d, N = layer->n_experts;
+  int rc = check_sizes(d, N, T, k);
+  if (rc) return rc;
+  if ((rc = check_dtype(x_dtype))) return rc;
+  if (T == 0) return ok();
+  if (!layer->w_packed || !layer->theta || !layer->phi || !x_host || !y_host || !w_gate)
+    return fail(BFMOE_EINVAL, "moe_forward_host: NULL pointer");
+  const HostPlan hp = make_host_plan(d, N, T, k, x_dtype, chunk);
+  if (!ws) return fail(BFMOE_EWORKSPACE, "moe_forward_host: NULL workspace");
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(BFMOE_EWORKSPACE, "moe_forward_host: workspace must be 256-byte aligned");
+  if (ws_bytes < hp.total)
+    return fail(BFMOE_EWORKSPACE, "moe_forward_host: workspace has %zu bytes, needs %zu", ws_bytes, hp.total);
+  HostPipe* pipe = nullptr;
+  SideStream* ss = nullptr;
+  if ((rc = host_pipe(&pipe)) || (rc = side_stream(&ss))) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* W = static_cast<uint8_t*>(ws);
+  const bool bf16 = x_dtype == BFMOE_BF16;
+  const size_t row_bytes = static_cast<size_t>(d) * (bf16 ? 2 : 4);
+  uint8_t* x_dev = W + hp.x_dev;
+  uint8_t* y_dev = W + hp.y_dev;
+  int32_t* idx = reinterpret_cast<int32_t*>(W + hp.idx);
+  float* gates = reinterpret_cast<float*>(W + hp.gates);
+  int32_t* counts = reinterpret_cast<int32_t*>(W + hp.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(W + hp.offsets);
+  int32_t* rows = reinterpret_cast<int32_t*>(W + hp.rows);
+  uint8_t* Wm = W + hp.moe;
+  const Plan pc = make_plan(d, N, hp.chunk, k, x_dtype);
+  const uint8_t* xh = static_cast<const uint8_t*>(x_host);
+  uint8_t* yh = static_cast<uint8_t*>(y_host);
+
+  // the copy streams start after all earlier work on `stream` (so a previous
+  // call's buffers are free); the weight tables build on the side stream
+  cudaError_t e = cudaEventRecord(pipe->fork, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(pipe->in, pipe->fork, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(pipe->out, pipe->fork, 0);
+  if (e == cudaSuccess) e = cudaEventRecord(ss->fork, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_forward_host: fork");
+  rc = build_weight_tables(layer, bf16, pc, Wm, ss->stream);
+  if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return cuda_fail(e, "moe_forward_host: join record");
+  for (int c = 0; c < hp.nchunks && rc == BFMOE_OK; ++c) {
+    const int t0 = hp.start[c], Tc = hp.start[c + 1] - t0;
+    const size_t o = static_cast<size_t>(t0) * row_bytes, n = static_cast<size_t>(Tc) * row_bytes;
+    if ((e = cudaMemcpyAsync(x_dev + o, xh + o, n, cudaMemcpyHostToDevice, pipe->in)) != cudaSuccess ||
+        (e = cudaEventRecord(pipe->ev_in[c], pipe->in)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(s, pipe->ev_in[c], 0)) != cudaSuccess) {
+      rc = cuda_fail(e, "moe_forward_host: copy in");
+      break;
+    }
+    rc = bfmoe_router_topk(x_dev + o, x_dtype, Tc, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows,
+                           Wm + pc.fwd_end, pc.rt_end, stream);
+    if (c == 0 && (e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) rc = cuda_fail(e, "moe_forward_host: join");
+    if (rc) break;
+    rc = forward_body(layer, x_dev + o, bf16, Tc, k, idx, gates, rows, y_dev + o, make_plan(d, N, Tc, k, x_dtype), Wm,
+                      s);
+    if (rc) break;
+    if ((e = cudaEventRecord(pipe->ev_out[c], s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(pipe->out, pipe->ev_out[c], 0)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(yh + o, y_dev + o, n, cudaMemcpyDeviceToHost, pipe->out)) != cudaSuccess)
+      rc = cuda_fail(e, "moe_forward_host: copy out");
+  }
+  // join: later work on `stream` runs after every copy out (and the side
+  // stream's tables, joined above or here when no chunk ran)
+  if ((e = cudaEventRecord(pipe->done, pipe->out)) == cudaSuccess) e = cudaStreamWaitEvent(s, pipe->done, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
+  if (e == cudaSuccess && (e = cudaEventRecord(pipe->fork, pipe->in)) == cudaSuccess)
+    e = cudaStreamWaitEvent(s, pipe->fork, 0);
+  if (e != cudaSuccess && rc == BFMOE_OK) rc = cuda_fail(e, "moe_forward_host: final join");
+  return rc ? rc : ok();
 }
 
 size_t bfmoe_moe_workspace_size(int d, int n_experts, int T, int k, int x_dtype) {

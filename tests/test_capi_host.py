@@ -61,3 +61,30 @@ def test_binding_names_match_header():
     import ternary_butterfly_experts_b200 as B
     for n in capi.header_functions():
         assert hasattr(B, n), f"binding lacks {n}"
+
+
+def test_host_call_checks_before_any_launch(L):
+    n0 = L.bfmoe_launch_count()
+    lay = capi.BfmoeLayer(64, 4, 16, ctypes.c_float(0.1), 16, 16)
+    f = L.bfmoe_moe_forward_host
+    assert f(None, 16, 1, 300, 16, None, 2, 16, 0, 256, 1 << 30, None) == capi.BFMOE_EINVAL       # no layer
+    assert f(ctypes.byref(lay), 16, 1, 300, 16, None, 5, 16, 0, 256, 1 << 30, None) == capi.BFMOE_EINVAL  # k > N
+    assert f(ctypes.byref(lay), None, 1, 300, 16, None, 2, 16, 0, 256, 1 << 30, None) == capi.BFMOE_EINVAL
+    assert f(ctypes.byref(lay), 16, 1, 300, 16, None, 2, None, 0, 256, 1 << 30, None) == capi.BFMOE_EINVAL
+    assert f(ctypes.byref(lay), 16, 3, 300, 16, None, 2, 16, 0, 256, 1 << 30, None) == capi.BFMOE_EINVAL  # dtype
+    assert f(ctypes.byref(lay), 16, 1, 300, 16, None, 2, 16, 0, None, 0, None) == capi.BFMOE_EWORKSPACE
+    assert f(ctypes.byref(lay), 16, 1, 300, 16, None, 2, 16, 0, 256, 100, None) == capi.BFMOE_EWORKSPACE
+    assert f(ctypes.byref(lay), 16, 1, 300, 16, None, 2, 16, 0, 264, 1 << 30, None) == capi.BFMOE_EWORKSPACE
+    assert f(ctypes.byref(lay), 16, 1, 0, 16, None, 2, 16, 0, None, 0, None) == capi.BFMOE_OK  # T = 0: nothing to do
+    assert L.bfmoe_launch_count() == n0
+
+
+def test_host_workspace_size(L):
+    bf = capi.BFMOE_BF16
+    full = L.bfmoe_moe_host_workspace_size(512, 256, 16384, 2, bf, 0)
+    one = L.bfmoe_moe_workspace_size(512, 256, 8192, 2, bf)
+    # device x and y for all tokens plus one default chunk (T/2) of scratch
+    assert full >= 2 * 16384 * 512 * 2 + one and full % 256 == 0
+    assert L.bfmoe_moe_host_workspace_size(512, 256, 16384, 2, bf, 16384) > full  # one big chunk needs more
+    assert L.bfmoe_moe_host_workspace_size(500, 256, 16384, 2, bf, 0) == 0
+    assert L.bfmoe_moe_host_workspace_size(512, 4, 100, 5, bf, 0) == 0
