@@ -32,6 +32,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte-aligned address in a dynamic shared-memory array (the
+// swizzled TMA tiles need it).  Offsetting the array itself, rather than
+// rounding an integer address, keeps the result a shared-memory pointer, so
+// the compiler emits shared (not generic) loads and stores through it.
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* base) {
+  return base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------

@@ -79,7 +79,7 @@ __global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const 
   using Cfg = GemmTcCfg<BN, STAGES>;
   static_assert(2 * BN == 64 || 2 * BN == 128 || 2 * BN == 256 || 2 * BN == 512, "TMEM columns");
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint32_t* epi = reinterpret_cast<uint32_t*>(smem + STAGES * Cfg::STAGE_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES + Cfg::EPI_BYTES);
   uint64_t* empty = full + STAGES;

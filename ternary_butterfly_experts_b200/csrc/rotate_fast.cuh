@@ -611,12 +611,21 @@ __device__ __forceinline__ void post_rotate_rows_smem(const Tz* zs0, const float
 #pragma unroll
   for (int g = 0; g < G; ++g) to_layout2<E>(v[g], buf, lane);
   l2_fwd<Gm, G, Gm::P>(v, tq, lane);
+  // gate, round, and write each row with 16-byte stores: the row goes through
+  // the warp's transpose buffer in natural order first
+  constexpr int NCH = Gm::D * static_cast<int>(sizeof(Ts)) / 16;  // 16-byte chunks per row
+  Ts* row_buf = reinterpret_cast<Ts*>(buf);
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    Ts* dst = slot + static_cast<size_t>(m[g].row) * Gm::D + lane;
     const float gt = m[g].gate;
 #pragma unroll
-    for (int q = 0; q < E; ++q) dst[q * 32] = from_f32<Ts>(gt * v[g][q]);
+    for (int q = 0; q < E; ++q) row_buf[q * 32 + lane] = from_f32<Ts>(gt * v[g][q]);
+    __syncwarp();
+    uint4* dst = reinterpret_cast<uint4*>(slot + static_cast<size_t>(m[g].row) * Gm::D);
+    const uint4* src = reinterpret_cast<const uint4*>(row_buf);
+#pragma unroll
+    for (int c = lane; c < NCH; c += 32) dst[c] = src[c];
+    __syncwarp();
   }
 }
 

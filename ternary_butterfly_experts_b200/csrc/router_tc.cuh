@@ -94,7 +94,7 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
                                                            int32_t* __restrict__ chunk_counts) {
   using Cfg = RouterTcCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
