@@ -101,6 +101,24 @@ cudaError_t launch(const char* name, cudaStream_t s, F&& f) {
   return e;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel of the stream finishes; it waits for that kernel's
+// results with pdl_wait() before touching global memory.
+template <typename... KP, typename... A>
+void pdl_launch(void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
 int grid_for(long long work, int per_block, int cap) {
   long long g = (work + per_block - 1) / per_block;
   if (g < 1) g = 1;
@@ -297,9 +315,8 @@ struct PreRotateFast {
     }
     const int grid = staged_grid<E, T>((a.R + C::G - 1) / C::G, resident);
     return launch("pre_rotate", a.s, [&] {
-      kern<<<grid, C::THREADS, C::SMEM, a.s>>>(static_cast<const T*>(a.x), a.idx, a.rows,
-                                               reinterpret_cast<const float4*>(a.cs), a.R, a.k, a.N,
-                                               static_cast<T*>(a.out));
+      pdl_launch(kern, grid, C::THREADS, C::SMEM, a.s, static_cast<const T*>(a.x), a.idx, a.rows,
+                 reinterpret_cast<const float4*>(a.cs), a.R, a.k, a.N, static_cast<T*>(a.out));
     });
   }
   // bf16 path: x and X_rot in bf16; float32 path: float32
@@ -319,9 +336,8 @@ struct PostRotateFast {
     }
     const int grid = staged_grid<E, T>((a.R + C::G - 1) / C::G, resident);
     return launch("post_rotate", a.s, [&] {
-      kern<<<grid, C::THREADS, C::SMEM, a.s>>>(static_cast<const T*>(a.z), a.idx, a.gates, a.rows,
-                                               reinterpret_cast<const float4*>(a.cs), a.R, a.N,
-                                               static_cast<T*>(a.out));
+      pdl_launch(kern, grid, C::THREADS, C::SMEM, a.s, static_cast<const T*>(a.z), a.idx, a.gates, a.rows,
+                 reinterpret_cast<const float4*>(a.cs), a.R, a.N, static_cast<T*>(a.out));
     });
   }
   // bf16 path: Z and slots in bf16; float32 path: float32
@@ -356,7 +372,7 @@ cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const C
   const long long tiles = static_cast<long long>((R + kGemmBM - 1) / kGemmBM) * (d / BN);
   const int grid = static_cast<int>(std::min<long long>(tiles, sm_count()));
   return launch("ternary_gemm_tc", s, [&] {
-    ternary_gemm_tc_kernel<BN, STAGES><<<grid, kGemmThreads, Cfg::SMEM_BYTES, s>>>(ta, tb, tbh, z, R, d, alpha);
+    pdl_launch(ternary_gemm_tc_kernel<BN, STAGES>, grid, kGemmThreads, Cfg::SMEM_BYTES, s, ta, tb, tbh, z, R, d, alpha);
   });
 }
 
@@ -373,7 +389,8 @@ cudaError_t launch_router_tc_k(const CUtensorMap& tx, const CUtensorMap& tw, con
   }
   const int grid = (T + kGemmBM - 1) / kGemmBM;
   return launch("router_tc", s, [&] {
-    router_tc_kernel<BN, STAGES, K><<<grid, kRouterThreads, Cfg::SMEM_BYTES, s>>>(tx, tw, bias, T, d, N, idx, gates, cc);
+    pdl_launch(router_tc_kernel<BN, STAGES, K>, grid, kRouterThreads, Cfg::SMEM_BYTES, s, tx, tw, bias, T, d, N, idx,
+               gates, cc);
   });
 }
 
@@ -500,8 +517,9 @@ int forward_body(const bfmoe_layer* layer, const void* x, bool bf16, int T, int 
   e = launch("combine", s, [&] {
     const int g = grid_for(nv, 256, sm_count() * 16);
     if (bf16 && fast)
-      combine_kernel<__nv_bfloat16, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(slot), T, k,
-                                                                     d, static_cast<__nv_bfloat16*>(y));
+      pdl_launch(combine_kernel<__nv_bfloat16, __nv_bfloat16>, g, 256, 0, s,
+                 static_cast<const __nv_bfloat16*>(slot), static_cast<long long>(T), k, d,
+                 static_cast<__nv_bfloat16*>(y));
     else if (bf16)
       combine_kernel<float, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d,
                                                              static_cast<__nv_bfloat16*>(y));
@@ -735,7 +753,7 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
     if (!aligned16(x)) return fail(BFMOE_EINVAL, "router_topk: x must be 16-byte aligned");
     __nv_bfloat16* parts = reinterpret_cast<__nv_bfloat16*>(W + p.wg_parts);
     const long long nw = static_cast<long long>(N) * d;
-    e = launch("router_split", s, [&] { router_split_kernel<<<grid_for(nw, 256, 2048), 256, 0, s>>>(w_gate, nw, parts); });
+    e = launch("router_split", s, [&] { pdl_launch(router_split_kernel, grid_for(nw, 256, 2048), 256, 0, s, w_gate, nw, parts); });
     if (e != cudaSuccess) return cuda_fail(e, "router_topk: split");
     const int BN = N >= 128 ? 128 : (N > 32 ? 64 : (N > 16 ? 32 : 16));
     CUtensorMap tx, tw;
@@ -778,11 +796,11 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
     e = launch("bucket_count", s, [&] { bucket_count_kernel<<<nchunks, chunk, N * 4, s>>>(idx, R, N, cc); });
     if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket count");
   }
-  e = launch("bucket_scan", s, [&] { bucket_scan_kernel<<<(N + 31) / 32, 1024, 0, s>>>(cc, nchunks, N, totals); });
+  e = launch("bucket_scan", s, [&] { pdl_launch(bucket_scan_kernel, (N + 31) / 32, 1024, 0, s, cc, nchunks, N, totals); });
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scan");
   const size_t scatter_smem = ((N + 1) * 4 + 15) / 16 * 16 + static_cast<size_t>(N) * 32;
   e = launch("bucket_scatter", s, [&] {
-    bucket_scatter_kernel<<<nchunks, chunk, scatter_smem, s>>>(idx, R, N, cc, totals, counts, offsets, rows);
+    pdl_launch(bucket_scatter_kernel, nchunks, chunk, scatter_smem, s, idx, R, N, cc, totals, counts, offsets, rows);
   });
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scatter");
   return ok();

@@ -42,6 +42,8 @@ __global__ __launch_bounds__(1024) void bucket_count_kernel(const int32_t* __res
 __global__ __launch_bounds__(1024) void bucket_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int N,
                                                            int32_t* __restrict__ totals) {
   __shared__ int part[32][33];
+  pdl_wait();
+  pdl_trigger();
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int e = blockIdx.x * 32 + tx;
   const int per = (nchunks + 31) / 32;
@@ -128,6 +130,8 @@ __global__ __launch_bounds__(1024) void bucket_scatter_kernel(const int32_t* __r
   uint8_t* wcnt = scatter_smem + ((N + 1) * 4 + 15) / 16 * 16;       // [N][32]: rows of expert e in warp w
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   for (int q = tid; q < N * 8; q += blockDim.x) reinterpret_cast<uint32_t*>(wcnt)[q] = 0u;
+  pdl_wait();
+  pdl_trigger();
   block_exclusive_scan(totals, N, off);
   if (blockIdx.x == 0) {
     for (int e = tid; e <= N; e += blockDim.x) {

@@ -41,6 +41,17 @@ __device__ __forceinline__ uint8_t* smem_align1024(uint8_t* base) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel of its stream finishes.
+// pdl_wait() blocks until that kernel has completed and its memory is
+// visible (a no-op for an ordinary launch); everything before it touches
+// only this CTA's shared memory, tensor memory and barriers.  pdl_trigger()
+// lets the next kernel start launching.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

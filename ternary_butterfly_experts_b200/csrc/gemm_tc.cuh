@@ -113,6 +113,8 @@ __global__ __launch_bounds__(kGemmThreads, 1) void ternary_gemm_tc_kernel(const 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // X_rot comes from the previous kernel
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {

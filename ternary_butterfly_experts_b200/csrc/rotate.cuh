@@ -218,6 +218,8 @@ __global__ __launch_bounds__(256) void post_rotate_kernel(const float* __restric
 template <typename Ts, typename Tout>
 __global__ __launch_bounds__(256) void combine_kernel(const Ts* __restrict__ slot, long long T, int k, int d,
                                                       Tout* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int VEC = 16 / sizeof(Ts);
   const int dv = d / VEC;
   const long long n = T * dv;

@@ -508,6 +508,8 @@ template <int E, typename Tin, typename Tout>
 __global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS, StagedCfg<E, Tin>::MIN_BLOCKS) void pre_rotate_fast_kernel(
     const Tin* __restrict__ x, const int32_t* __restrict__ idx, const int32_t* __restrict__ rows,
     const float4* __restrict__ quads, long long R, int k, int N, Tout* __restrict__ xrot) {
+  pdl_wait();
+  pdl_trigger();
   using C = StagedCfg<E, Tin>;
   using Gm = typename C::Gm;
   constexpr int G = C::G, D = Gm::D;
@@ -635,6 +637,8 @@ template <int E, typename Tz, typename Ts>
 __global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS, StagedCfg<E, Tz>::MIN_BLOCKS) void post_rotate_fast_kernel(
     const Tz* __restrict__ z, const int32_t* __restrict__ idx, const float* __restrict__ gates,
     const int32_t* __restrict__ rows, const float4* __restrict__ quads, long long R, int N, Ts* __restrict__ slot) {
+  pdl_wait();
+  pdl_trigger();
   using C = StagedCfg<E, Tz>;
   using Gm = typename C::Gm;
   constexpr int G = C::G, D = Gm::D;

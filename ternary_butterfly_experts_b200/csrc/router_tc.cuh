@@ -27,6 +27,8 @@ namespace bfmoe {
 
 // w [N][d] float32 -> parts [3][N][d] bfloat16 with hi + mid + lo == w.
 __global__ void router_split_kernel(const float* __restrict__ w, long long n, __nv_bfloat16* __restrict__ parts) {
+  pdl_wait();
+  pdl_trigger();
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const float v = w[i];
@@ -133,6 +135,8 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the split weights come from the previous kernel
+  pdl_trigger();
 
   if (warp == 0 && lane == 0) {
     int it = 0;
