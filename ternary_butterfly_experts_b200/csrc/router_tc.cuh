@@ -70,8 +70,11 @@ struct TopK {
       id[j] = 0x7fffffff;
     }
   }
+  // Small K: the K compare-and-select steps run for every column, with no
+  // branch (the lanes of a warp hold different rows, so an early exit would
+  // diverge on most columns); larger K exits first when l cannot enter.
   __device__ __forceinline__ void push(float l, int e) {
-    if (!ranks_before(l, e, v[K - 1], id[K - 1])) return;
+    if (K > 4 && !ranks_before(l, e, v[K - 1], id[K - 1])) return;
     float cv = l;
     int ci = e;
 #pragma unroll
