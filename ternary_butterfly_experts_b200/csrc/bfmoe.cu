@@ -119,6 +119,22 @@ void pdl_launch(void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cudaStr
   cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
 }
 
+// Kernel attributes (dynamic shared-memory limits) are set per device: the
+// first launch of a kernel on each device sets them.  `done` holds one bit
+// per device and is set only after the attribute, so concurrent first calls
+// both set it (the call is idempotent).
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev & 63;
+}
+bool needs_attr(const std::atomic<uint64_t>& done) {
+  return (done.load(std::memory_order_acquire) >> current_device() & 1u) == 0;
+}
+void attr_set(std::atomic<uint64_t>& done) {
+  done.fetch_or(uint64_t(1) << current_device(), std::memory_order_release);
+}
+
 int grid_for(long long work, int per_block, int cap) {
   long long g = (work + per_block - 1) / per_block;
   if (g < 1) g = 1;
@@ -126,15 +142,19 @@ int grid_for(long long work, int per_block, int cap) {
   return static_cast<int>(g);
 }
 
+// SMs of the current device (cached per device).
 int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  static std::atomic<int> n[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  int v = n[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (v <= 0) v = 148;
+    n[dev].store(v, std::memory_order_relaxed);
   }
-  return n;
+  return v;
 }
 
 // ---------------------------------------------------------------------------
@@ -308,12 +328,15 @@ struct PreRotateFast {
   static cudaError_t go(const RotArgs& a) {
     using C = StagedCfg<E, T>;
     auto kern = pre_rotate_fast_kernel<E, T, T>;
-    static int resident = 0;
-    if (resident == 0) {
+    static std::atomic<uint64_t> done{0};
+    static int resident[64] = {};
+    const int dev = current_device();
+    if (needs_attr(done)) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
-      resident = resident_ctas(kern, C::THREADS, C::SMEM);
+      resident[dev] = resident_ctas(kern, C::THREADS, C::SMEM);
+      attr_set(done);
     }
-    const int grid = staged_grid<E, T>((a.R + C::G - 1) / C::G, resident);
+    const int grid = staged_grid<E, T>((a.R + C::G - 1) / C::G, resident[dev]);
     return launch("pre_rotate", a.s, [&] {
       pdl_launch(kern, grid, C::THREADS, C::SMEM, a.s, static_cast<const T*>(a.x), a.idx, a.rows,
                  reinterpret_cast<const float4*>(a.cs), a.R, a.k, a.N, static_cast<T*>(a.out));
@@ -329,12 +352,15 @@ struct PostRotateFast {
   static cudaError_t go(const RotArgs& a) {
     using C = StagedCfg<E, T>;
     auto kern = post_rotate_fast_kernel<E, T, T>;
-    static int resident = 0;
-    if (resident == 0) {
+    static std::atomic<uint64_t> done{0};
+    static int resident[64] = {};
+    const int dev = current_device();
+    if (needs_attr(done)) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM));
-      resident = resident_ctas(kern, C::THREADS, C::SMEM);
+      resident[dev] = resident_ctas(kern, C::THREADS, C::SMEM);
+      attr_set(done);
     }
-    const int grid = staged_grid<E, T>((a.R + C::G - 1) / C::G, resident);
+    const int grid = staged_grid<E, T>((a.R + C::G - 1) / C::G, resident[dev]);
     return launch("post_rotate", a.s, [&] {
       pdl_launch(kern, grid, C::THREADS, C::SMEM, a.s, static_cast<const T*>(a.z), a.idx, a.gates, a.rows,
                  reinterpret_cast<const float4*>(a.cs), a.R, a.N, static_cast<T*>(a.out));
@@ -362,12 +388,12 @@ template <int BN, int STAGES>
 cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tbh, __nv_bfloat16* z,
                            int R, int d, float alpha, cudaStream_t s) {
   using Cfg = GemmTcCfg<BN, STAGES>;
-  static bool attr = false;
-  if (!attr) {
+  static std::atomic<uint64_t> done{0};
+  if (needs_attr(done)) {
     cudaError_t e = cudaFuncSetAttribute(ternary_gemm_tc_kernel<BN, STAGES>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr_set(done);
   }
   const long long tiles = static_cast<long long>((R + kGemmBM - 1) / kGemmBM) * (d / BN);
   const int grid = static_cast<int>(std::min<long long>(tiles, sm_count()));
@@ -380,12 +406,12 @@ template <int BN, int STAGES, int K>
 cudaError_t launch_router_tc_k(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
                                int32_t* idx, float* gates, int32_t* cc, cudaStream_t s) {
   using Cfg = RouterTcCfg<BN, STAGES>;
-  static bool attr = false;
-  if (!attr) {
+  static std::atomic<uint64_t> done{0};
+  if (needs_attr(done)) {
     cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<BN, STAGES, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr_set(done);
   }
   const int grid = (T + kGemmBM - 1) / kGemmBM;
   return launch("router_tc", s, [&] {
@@ -442,11 +468,11 @@ int build_weight_tables(const bfmoe_layer* layer, bool bf16, const Plan& p, uint
     const int tab_blocks = 2 * N;
     const int exp_blocks = bf16 ? grid_for(static_cast<long long>(d) * (d / 16), 256, 1024) : 0;
     const size_t tab_smem = static_cast<size_t>(L) * d * sizeof(float);  // cos and sin of one expert
-    static bool tab_attr = false;
-    if (!tab_attr) {
+    static std::atomic<uint64_t> done{0};
+    if (needs_attr(done)) {
       cudaFuncSetAttribute(rot_quads_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(12 * BFMOE_MAX_D * sizeof(float)));
-      tab_attr = true;
+      attr_set(done);
     }
     e = launch("rot_table", s, [&] {
       rot_quads_kernel<<<tab_blocks + exp_blocks, 256, tab_smem, s>>>(
@@ -785,12 +811,12 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
 
   const int chunk = bucket_chunk(k);
   const int nchunks = static_cast<int>((R + chunk - 1) / chunk);
-  static bool attr = false;
-  if (!attr) {
+  static std::atomic<uint64_t> done{0};
+  if (needs_attr(done)) {
     cudaFuncSetAttribute(bucket_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BFMOE_MAX_EXPERTS * 4);
     cudaFuncSetAttribute(bucket_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          BFMOE_MAX_EXPERTS * 36 + 16);
-    attr = true;
+    attr_set(done);
   }
   if (!tc_router) {  // the tensor-core router writes the chunk histograms itself
     e = launch("bucket_count", s, [&] { bucket_count_kernel<<<nchunks, chunk, N * 4, s>>>(idx, R, N, cc); });

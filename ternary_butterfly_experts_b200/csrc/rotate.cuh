@@ -121,7 +121,22 @@ __device__ __forceinline__ void load_row(const T* __restrict__ src, float (&v)[E
 template <int E, typename T>
 __device__ __forceinline__ void store_row(T* __restrict__ dst, const float (&v)[E], bool active) {
   if (!active) return;
-  if constexpr ((E * sizeof(T)) % 16 == 0) {
+  if constexpr ((E * sizeof(T)) % 32 == 0) {
+    // 32 bytes per store: one whole L2 sector per lane (dst is 32-byte aligned:
+    // rows of 32*E elements in a 256-byte aligned workspace)
+    constexpr int NV = E * sizeof(T) / 32;
+    constexpr int PER = 32 / sizeof(T);
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+      uint32_t w[8];
+      T* p = reinterpret_cast<T*>(w);
+#pragma unroll
+      for (int q = 0; q < PER; ++q) p[q] = from_f32<T>(v[u * PER + q]);
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + u * PER), "r"(w[0]),
+                   "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                   : "memory");
+    }
+  } else if constexpr ((E * sizeof(T)) % 16 == 0) {
     constexpr int NV = E * sizeof(T) / 16;
     constexpr int PER = 16 / sizeof(T);
 #pragma unroll
