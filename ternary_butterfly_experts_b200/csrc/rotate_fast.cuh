@@ -429,9 +429,16 @@ struct StagedCfg {
   static constexpr size_t TAB_QUADS = tab_quads(E);
   static constexpr int MIN_BLOCKS = E <= 32 ? 2 : 1;
   static constexpr int MAXJ = 32 / G;  // groups per warp (one row's metadata per lane)
-  // per warp: two buffers of G staged rows and one float32 transpose buffer
+  // per warp: two buffers of G staged rows, and a float32 transpose buffer.
+  // Once a group's rows are in registers its staging buffer is free until
+  // the group after next is fetched, so the transpose buffer lives there when
+  // it fits; the shared memory saved is left to L1, which holds the cos/sin
+  // tables.
   static constexpr size_t BUF_BYTES = G * Gm::D * sizeof(Tin);
-  static constexpr size_t WARP_BYTES = 2 * BUF_BYTES + Gm::D * 4;
+  // (at d = 512 the tables fit in L1 anyway, and the register-resident group
+  // walk below costs spills there: 33 -> 36 us pre, 37 -> 47 us post)
+  static constexpr bool TBUF_IN_STAGE = E >= 32 && BUF_BYTES >= Gm::D * 4;
+  static constexpr size_t WARP_BYTES = 2 * BUF_BYTES + (TBUF_IN_STAGE ? 0 : Gm::D * 4);
   static constexpr size_t SMEM = Gm::WARPS * WARP_BYTES;
 };
 
@@ -485,21 +492,43 @@ __device__ __forceinline__ RowMeta shfl_meta(const RowMeta& m, int src) {
                  __shfl_sync(FULL_MASK, m.gate, src)};
 }
 
-template <class Gm, int G, typename Tin, typename Tout>
-__device__ __forceinline__ void pre_rotate_rows_smem(const Tin* xs0, const float4* tq, Tout* __restrict__ dst0,
-                                                     float* buf, int lane) {
-  constexpr int E = Gm::E;
-  float v[G][E];
+// G staged rows (natural order) into registers, layout 2.
+template <class Gm, int G, typename Tin>
+__device__ __forceinline__ void load_rows_l2(const Tin* xs0, float (&v)[G][Gm::E], int lane) {
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int q = 0; q < E; ++q) v[g][q] = to_f32(xs0[g * Gm::D + q * 32 + lane]);  // layout 2
+    for (int q = 0; q < Gm::E; ++q) v[g][q] = to_f32(xs0[g * Gm::D + q * 32 + lane]);
+}
+
+template <class Gm, int G, typename Tout>
+__device__ __forceinline__ void pre_rotate_regs(float (&v)[G][Gm::E], const float4* tq, Tout* __restrict__ dst0,
+                                                float* buf, int lane) {
+  constexpr int E = Gm::E;
   l2_tr<Gm, G, Gm::L - 1>(v, tq, lane);
 #pragma unroll
   for (int g = 0; g < G; ++g) to_layout1<E>(v[g], buf, lane);
   l1_tr<Gm, G, Gm::P - 1>(v, tq, lane);
 #pragma unroll
   for (int g = 0; g < G; ++g) store_row<E, Tout>(dst0 + static_cast<size_t>(g) * Gm::D + lane * E, v[g], true);
+}
+
+template <class Gm, int G, typename Tin, typename Tout>
+__device__ __forceinline__ void pre_rotate_rows_smem(const Tin* xs0, const float4* tq, Tout* __restrict__ dst0,
+                                                     float* buf, int lane) {
+  float v[G][Gm::E];
+  load_rows_l2<Gm, G, Tin>(xs0, v, lane);
+  pre_rotate_regs<Gm, G, Tout>(v, tq, dst0, buf, lane);
+}
+
+// Row 0 of v <- row 1 <- ... (static register moves), for walking a group
+// row by row without indexing the register array.
+template <int G, int E>
+__device__ __forceinline__ void shift_rows(float (&v)[G][E]) {
+#pragma unroll
+  for (int h = 0; h + 1 < G; ++h)
+#pragma unroll
+    for (int q = 0; q < E; ++q) v[h][q] = v[h + 1][q];
 }
 
 // xrot[p] = B(theta_e)^T x_t for bucket positions p (row r = rows[p],
@@ -524,7 +553,7 @@ __global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS, StagedCfg<E, Tin>::MIN_
   }
   uint8_t* wbase = smem_raw + w * C::WARP_BYTES;
   Tin* xs = reinterpret_cast<Tin*>(wbase);
-  float* buf = reinterpret_cast<float*>(wbase + 2 * C::BUF_BYTES);
+  float* tbuf = reinterpret_cast<float*>(wbase + 2 * C::BUF_BYTES);
   auto pos0 = [&](int j) { return (wg.gb0 + w + static_cast<long long>(Gm::WARPS) * j) * G; };
 
   const int jl = lane / G;
@@ -555,41 +584,69 @@ __global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS, StagedCfg<E, Tin>::MIN_
       cp_async_wait<0>();
     }
     __syncwarp();
-    const Tin* cur = xs + (j & 1) * G * D;
+    Tin* cur = xs + (j & 1) * G * D;
     const long long p0 = pos0(j);
     const int e0 = __shfl_sync(FULL_MASK, mine.ex, j * G);
     const unsigned gm = ((1u << G) - 1u) << (j * G);
     const unsigned same = __ballot_sync(FULL_MASK, mine.ex >= 0 && mine.ex == e0) & gm;
-    if (same == gm && p0 + G <= R) {
-      pre_rotate_rows_smem<Gm, G, Tin, Tout>(cur, quads + static_cast<size_t>(e0) * C::TAB_QUADS, xrot + p0 * D,
-                                             buf, lane);
-    } else {
+    if constexpr (C::TBUF_IN_STAGE) {
+      // the whole group goes to registers first; its staging buffer then
+      // serves as the transpose buffer, and a mixed group is walked row by
+      // row in registers
+      float* buf = reinterpret_cast<float*>(cur);
+      float v[G][E];
+      load_rows_l2<Gm, G, Tin>(cur, v, lane);
+      __syncwarp();  // all lanes have read the staged rows before buf (which aliases them) is written
+      if (same == gm && p0 + G <= R) {
+        pre_rotate_regs<Gm, G, Tout>(v, quads + static_cast<size_t>(e0) * C::TAB_QUADS, xrot + p0 * D, buf, lane);
+      } else {
 #pragma unroll 1
-      for (int g = 0; g < G; ++g) {
-        const long long p = p0 + g;
-        if (p >= R) break;
-        const int e = __shfl_sync(FULL_MASK, mine.ex, j * G + g);
-        if (e < 0) {
-          float z[E];
+        for (int g = 0; g < G; ++g) {
+          const long long p = p0 + g;
+          if (p >= R) break;
+          const int e = __shfl_sync(FULL_MASK, mine.ex, j * G + g);
+          float v1[1][E];
 #pragma unroll
-          for (int q = 0; q < E; ++q) z[q] = 0.f;
-          store_row<E, Tout>(xrot + p * D + lane * E, z, true);
-          continue;
+          for (int q = 0; q < E; ++q) v1[0][q] = e < 0 ? 0.f : v[0][q];
+          if (e < 0) {
+            store_row<E, Tout>(xrot + p * D + lane * E, v1[0], true);
+          } else {
+            pre_rotate_regs<Gm, 1, Tout>(v1, quads + static_cast<size_t>(e) * C::TAB_QUADS, xrot + p * D, buf, lane);
+          }
+          shift_rows<G, E>(v);
         }
-        pre_rotate_rows_smem<Gm, 1, Tin, Tout>(cur + g * D, quads + static_cast<size_t>(e) * C::TAB_QUADS,
-                                               xrot + p * D, buf, lane);
+      }
+    } else {
+      if (same == gm && p0 + G <= R) {
+        pre_rotate_rows_smem<Gm, G, Tin, Tout>(cur, quads + static_cast<size_t>(e0) * C::TAB_QUADS, xrot + p0 * D,
+                                               tbuf, lane);
+      } else {
+#pragma unroll 1
+        for (int g = 0; g < G; ++g) {
+          const long long p = p0 + g;
+          if (p >= R) break;
+          const int e = __shfl_sync(FULL_MASK, mine.ex, j * G + g);
+          if (e < 0) {
+            float z[E];
+#pragma unroll
+            for (int q = 0; q < E; ++q) z[q] = 0.f;
+            store_row<E, Tout>(xrot + p * D + lane * E, z, true);
+            continue;
+          }
+          pre_rotate_rows_smem<Gm, 1, Tin, Tout>(cur + g * D, quads + static_cast<size_t>(e) * C::TAB_QUADS,
+                                                 xrot + p * D, tbuf, lane);
+        }
       }
     }
     __syncwarp();  // buffer j & 1 is refilled by issue(j + 2)
   }
 }
 
-template <class Gm, int G, typename Tz, typename Ts>
-__device__ __forceinline__ void post_rotate_rows_smem(const Tz* zs0, const float4* tq, const RowMeta* m,
-                                                      Ts* __restrict__ slot, float* buf, int lane) {
+// G staged rows (16-byte chunks swizzled by chunk_swz) into registers, layout 1.
+template <class Gm, int G, typename Tz>
+__device__ __forceinline__ void load_rows_l1(const Tz* zs0, float (&v)[G][Gm::E], int lane) {
   constexpr int E = Gm::E;
   constexpr int PER = 16 / sizeof(Tz);  // elements per 16-byte chunk
-  float v[G][E];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const uint8_t* zr = reinterpret_cast<const uint8_t*>(zs0 + g * Gm::D);
@@ -609,6 +666,12 @@ __device__ __forceinline__ void post_rotate_rows_smem(const Tz* zs0, const float
       }
     }
   }
+}
+
+template <class Gm, int G, typename Ts>
+__device__ __forceinline__ void post_rotate_regs(float (&v)[G][Gm::E], const float4* tq, const RowMeta* m,
+                                                 Ts* __restrict__ slot, float* buf, int lane) {
+  constexpr int E = Gm::E;
   l1_fwd<Gm, G, 0>(v, tq, lane);
 #pragma unroll
   for (int g = 0; g < G; ++g) to_layout2<E>(v[g], buf, lane);
@@ -629,6 +692,14 @@ __device__ __forceinline__ void post_rotate_rows_smem(const Tz* zs0, const float
     for (int c = lane; c < NCH; c += 32) dst[c] = src[c];
     __syncwarp();
   }
+}
+
+template <class Gm, int G, typename Tz, typename Ts>
+__device__ __forceinline__ void post_rotate_rows_smem(const Tz* zs0, const float4* tq, const RowMeta* m,
+                                                      Ts* __restrict__ slot, float* buf, int lane) {
+  float v[G][Gm::E];
+  load_rows_l1<Gm, G, Tz>(zs0, v, lane);
+  post_rotate_regs<Gm, G, Ts>(v, tq, m, slot, buf, lane);
 }
 
 // slot[r] = g_r * B(phi_e) z_p for bucket positions p (z already scaled by
@@ -653,7 +724,7 @@ __global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS, StagedCfg<E, Tz>::MIN_BL
   }
   uint8_t* wbase = smem_raw + w * C::WARP_BYTES;
   Tz* zs = reinterpret_cast<Tz*>(wbase);
-  float* buf = reinterpret_cast<float*>(wbase + 2 * C::BUF_BYTES);
+  float* tbuf = reinterpret_cast<float*>(wbase + 2 * C::BUF_BYTES);
   auto pos0 = [&](int j) { return (wg.gb0 + w + static_cast<long long>(Gm::WARPS) * j) * G; };
 
   const int jl = lane / G;
@@ -684,24 +755,53 @@ __global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS, StagedCfg<E, Tz>::MIN_BL
       cp_async_wait<0>();
     }
     __syncwarp();
-    const Tz* cur = zs + (j & 1) * G * D;
+    Tz* cur = zs + (j & 1) * G * D;
     const long long p0 = pos0(j);
     const int e0 = __shfl_sync(FULL_MASK, mine.ex, j * G);
     const unsigned gm = ((1u << G) - 1u) << (j * G);
     const unsigned same = __ballot_sync(FULL_MASK, mine.ex >= 0 && mine.ex == e0) & gm;
-    if (same == gm && p0 + G <= R) {
-      RowMeta m[G];
+    if constexpr (C::TBUF_IN_STAGE) {
+      // as in the pre-rotation: group in registers, staging buffer reused
+      float* buf = reinterpret_cast<float*>(cur);
+      float v[G][E];
+      load_rows_l1<Gm, G, Tz>(cur, v, lane);
+      __syncwarp();  // all lanes have read the staged rows before buf (which aliases them) is written
+      if (same == gm && p0 + G <= R) {
+        RowMeta m[G];
 #pragma unroll
-      for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, j * G + g);
-      post_rotate_rows_smem<Gm, G, Tz, Ts>(cur, quads + static_cast<size_t>(e0) * C::TAB_QUADS, m, slot, buf, lane);
-    } else {
+        for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, j * G + g);
+        post_rotate_regs<Gm, G, Ts>(v, quads + static_cast<size_t>(e0) * C::TAB_QUADS, m, slot, buf, lane);
+      } else {
 #pragma unroll 1
-      for (int g = 0; g < G; ++g) {
-        if (p0 + g >= R) break;
-        const RowMeta m1[1] = {shfl_meta(mine, j * G + g)};
-        if (m1[0].ex < 0) continue;
-        post_rotate_rows_smem<Gm, 1, Tz, Ts>(cur + g * D, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS, m1,
-                                             slot, buf, lane);
+        for (int g = 0; g < G; ++g) {
+          if (p0 + g >= R) break;
+          const RowMeta m1[1] = {shfl_meta(mine, j * G + g)};
+          if (m1[0].ex >= 0) {
+            float v1[1][E];
+#pragma unroll
+            for (int q = 0; q < E; ++q) v1[0][q] = v[0][q];
+            post_rotate_regs<Gm, 1, Ts>(v1, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS, m1, slot, buf,
+                                        lane);
+          }
+          shift_rows<G, E>(v);
+        }
+      }
+    } else {
+      if (same == gm && p0 + G <= R) {
+        RowMeta m[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, j * G + g);
+        post_rotate_rows_smem<Gm, G, Tz, Ts>(cur, quads + static_cast<size_t>(e0) * C::TAB_QUADS, m, slot, tbuf,
+                                             lane);
+      } else {
+#pragma unroll 1
+        for (int g = 0; g < G; ++g) {
+          if (p0 + g >= R) break;
+          const RowMeta m1[1] = {shfl_meta(mine, j * G + g)};
+          if (m1[0].ex < 0) continue;
+          post_rotate_rows_smem<Gm, 1, Tz, Ts>(cur + g * D, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS,
+                                               m1, slot, tbuf, lane);
+        }
       }
     }
     __syncwarp();  // buffer j & 1 is refilled by issue(j + 2)

@@ -126,6 +126,27 @@ def test_large_workloads_sampled(name):
     assert np.array_equal(np.diff(gpu["offsets"]), gpu["counts"])
 
 
+# -- the boundary's maximum sizes ------------------------------------------------------
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_maximum_d(dt):
+    """d = 4096, the largest d the boundary accepts: 12 stages, one row per warp."""
+    wl = W.custom("dmax", d=4096, n_experts=4, k=2, tokens=37, dtype=dt, bias_var=0.5)
+    inp = W.generate(wl, seed=11)
+    gpu = run_cuda(inp)
+    c, o, r = O.buckets(gpu["idx"], wl.n_experts)
+    assert np.array_equal(gpu["counts"], c) and np.array_equal(gpu["offsets"], o)
+    assert np.array_equal(gpu["rows"], r)
+    compare(inp, gpu, tokens=np.arange(wl.tokens))
+
+
+def test_maximum_experts_and_k():
+    """N = 4096 experts (the boundary's limit) with k = 8, the largest top-k."""
+    wl = W.custom("nmax", d=64, n_experts=4096, k=8, tokens=300, dtype="bf16", bias_var=0.5)
+    inp = W.generate(wl, seed=12)
+    compare(inp, run_cuda(inp))
+
+
 # -- edge cases ---------------------------------------------------------------------
 
 def test_single_token_and_single_expert():
