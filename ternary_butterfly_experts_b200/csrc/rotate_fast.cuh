@@ -443,13 +443,17 @@ struct StagedCfg {
 };
 
 // Grid for `groups` groups when `resident` CTAs fit on the device at once.
+// A warp takes at most MAXJ groups, so `need` CTAs at least; the grid is a
+// whole number of full waves of `resident` CTAs (no partly filled last wave),
+// and no larger than one group per warp.
 template <int E, typename Tin>
 __host__ inline int staged_grid(long long groups, int resident) {
   using C = StagedCfg<E, Tin>;
   const long long per = static_cast<long long>(C::Gm::WARPS);
+  const long long res = resident > 0 ? resident : 1;
   long long g = (groups + per - 1) / per;                               // one group per warp at most
   const long long need = (groups + per * C::MAXJ - 1) / (per * C::MAXJ);  // MAXJ groups per warp at least
-  const long long want = resident > need ? resident : need;
+  const long long want = (need + res - 1) / res * res;
   if (g > want) g = want;
   return static_cast<int>(g < 1 ? 1 : g);
 }
