@@ -350,7 +350,7 @@ template <int E>
 struct PostRotateFast {
   template <typename T>
   static cudaError_t go(const RotArgs& a) {
-    using C = StagedCfg<E, T>;
+    using C = StagedCfg<E, T, false>;
     auto kern = post_rotate_fast_kernel<E, T, T>;
     static std::atomic<uint64_t> done{0};
     static int resident[64] = {};
@@ -360,7 +360,7 @@ struct PostRotateFast {
       resident[dev] = resident_ctas(kern, C::THREADS, C::SMEM);
       attr_set(done);
     }
-    const int grid = staged_grid<E, T>((a.R + C::G - 1) / C::G, resident[dev]);
+    const int grid = staged_grid<E, T, false>((a.R + C::G - 1) / C::G, resident[dev]);
     return launch("post_rotate", a.s, [&] {
       pdl_launch(kern, grid, C::THREADS, C::SMEM, a.s, static_cast<const T*>(a.z), a.idx, a.gates, a.rows,
                  reinterpret_cast<const float4*>(a.cs), a.R, a.N, static_cast<T*>(a.out));

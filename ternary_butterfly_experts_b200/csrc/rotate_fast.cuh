@@ -395,6 +395,63 @@ __device__ __forceinline__ void to_layout1(float (&r)[E], float* buf, int lane) 
   __syncwarp();
 }
 
+// The same switches through a buffer of only D/2 floats, one half of the row
+// at a time.  Half h of the elements (indices [h*16E, (h+1)*16E)) is held by
+// lanes 16h..16h+15 in layout 1 and by registers [h*E/2, (h+1)*E/2) of every
+// lane in layout 2; t keeps the values that the first pass moved until the
+// second pass no longer needs the registers they land in.
+template <int E>
+__device__ __forceinline__ void to_layout2_halves(float (&r)[E], float* buf, int lane) {
+  static_assert(E >= 8, "vector stores of four");
+  constexpr int H = E / 2;
+  float t[H];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if ((lane >> 4) == h) {
+#pragma unroll
+      for (int u = 0; u < E / 4; ++u) {
+        const int i = (lane & 15) * E + 4 * u;
+        *reinterpret_cast<float4*>(buf + swz(i)) = make_float4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < H; ++q) {
+      const float val = buf[swz(q * 32 + lane)];
+      if (h == 0) t[q] = val; else r[H + q] = val;
+    }
+    __syncwarp();
+  }
+#pragma unroll
+  for (int q = 0; q < H; ++q) r[q] = t[q];
+}
+
+template <int E>
+__device__ __forceinline__ void to_layout1_halves(float (&r)[E], float* buf, int lane) {
+  static_assert(E >= 8, "vector loads of four");
+  constexpr int H = E / 2;
+  float t[H];
+#pragma unroll
+  for (int q = 0; q < H; ++q) t[q] = r[H + q];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int q = 0; q < H; ++q) buf[swz(q * 32 + lane)] = h == 0 ? r[q] : t[q];
+    __syncwarp();
+    if ((lane >> 4) == h) {
+#pragma unroll
+      for (int u = 0; u < E / 4; ++u) {
+        const float4 v4 = *reinterpret_cast<const float4*>(buf + swz((lane & 15) * E + 4 * u));
+        r[4 * u] = v4.x;
+        r[4 * u + 1] = v4.y;
+        r[4 * u + 2] = v4.z;
+        r[4 * u + 3] = v4.w;
+      }
+    }
+    __syncwarp();
+  }
+}
+
 // ---- kernels: persistent warps, rows double-buffered in shared memory ----------
 //
 // The bucket positions are cut into groups of G consecutive positions.  The
@@ -421,7 +478,10 @@ __device__ __forceinline__ void cp_async_wait() {
 // reads of 8 lanes then hit 8 different bank groups.
 __device__ __forceinline__ int chunk_swz(int c) { return c ^ ((c >> 3) & 7); }
 
-template <int E, typename Tin>
+// HALVES: whether a staging buffer of half a float32 row may hold the
+// transpose buffer (layout switches in two halves); the pre-rotation gains
+// from it at d = 2048 (2775 -> 2512 us), the post-rotation does not.
+template <int E, typename Tin, bool HALVES = true>
 struct StagedCfg {
   using Gm = Geo<E>;
   static constexpr int G = Gm::G;
@@ -437,7 +497,9 @@ struct StagedCfg {
   static constexpr size_t BUF_BYTES = G * Gm::D * sizeof(Tin);
   // (at d = 512 the tables fit in L1 anyway, and the register-resident group
   // walk below costs spills there: 33 -> 36 us pre, 37 -> 47 us post)
-  static constexpr bool TBUF_IN_STAGE = E >= 32 && BUF_BYTES >= Gm::D * 4;
+  static constexpr bool TBUF_IN_STAGE = E >= 32 && E <= 64 && BUF_BYTES >= Gm::D * (HALVES ? 2 : 4);
+  // a staging buffer of half a float32 row (one bf16 row) switches layouts in halves
+  static constexpr bool TBUF_HALVES = TBUF_IN_STAGE && BUF_BYTES < Gm::D * 4;
   static constexpr size_t WARP_BYTES = 2 * BUF_BYTES + (TBUF_IN_STAGE ? 0 : Gm::D * 4);
   static constexpr size_t SMEM = Gm::WARPS * WARP_BYTES;
 };
@@ -446,9 +508,9 @@ struct StagedCfg {
 // A warp takes at most MAXJ groups, so `need` CTAs at least; the grid is a
 // whole number of full waves of `resident` CTAs (no partly filled last wave),
 // and no larger than one group per warp.
-template <int E, typename Tin>
+template <int E, typename Tin, bool HALVES = true>
 __host__ inline int staged_grid(long long groups, int resident) {
-  using C = StagedCfg<E, Tin>;
+  using C = StagedCfg<E, Tin, HALVES>;
   const long long per = static_cast<long long>(C::Gm::WARPS);
   const long long res = resident > 0 ? resident : 1;
   long long g = (groups + per - 1) / per;                               // one group per warp at most
@@ -505,13 +567,16 @@ __device__ __forceinline__ void load_rows_l2(const Tin* xs0, float (&v)[G][Gm::E
     for (int q = 0; q < Gm::E; ++q) v[g][q] = to_f32(xs0[g * Gm::D + q * 32 + lane]);
 }
 
-template <class Gm, int G, typename Tout>
+template <class Gm, int G, typename Tout, bool HALVES = false>
 __device__ __forceinline__ void pre_rotate_regs(float (&v)[G][Gm::E], const float4* tq, Tout* __restrict__ dst0,
                                                 float* buf, int lane) {
   constexpr int E = Gm::E;
   l2_tr<Gm, G, Gm::L - 1>(v, tq, lane);
 #pragma unroll
-  for (int g = 0; g < G; ++g) to_layout1<E>(v[g], buf, lane);
+  for (int g = 0; g < G; ++g) {
+    if constexpr (HALVES) to_layout1_halves<E>(v[g], buf, lane);
+    else to_layout1<E>(v[g], buf, lane);
+  }
   l1_tr<Gm, G, Gm::P - 1>(v, tq, lane);
 #pragma unroll
   for (int g = 0; g < G; ++g) store_row<E, Tout>(dst0 + static_cast<size_t>(g) * Gm::D + lane * E, v[g], true);
@@ -602,7 +667,7 @@ __global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS, StagedCfg<E, Tin>::MIN_
       load_rows_l2<Gm, G, Tin>(cur, v, lane);
       __syncwarp();  // all lanes have read the staged rows before buf (which aliases them) is written
       if (same == gm && p0 + G <= R) {
-        pre_rotate_regs<Gm, G, Tout>(v, quads + static_cast<size_t>(e0) * C::TAB_QUADS, xrot + p0 * D, buf, lane);
+        pre_rotate_regs<Gm, G, Tout, C::TBUF_HALVES>(v, quads + static_cast<size_t>(e0) * C::TAB_QUADS, xrot + p0 * D, buf, lane);
       } else {
 #pragma unroll 1
         for (int g = 0; g < G; ++g) {
@@ -615,7 +680,7 @@ __global__ __launch_bounds__(StagedCfg<E, Tin>::THREADS, StagedCfg<E, Tin>::MIN_
           if (e < 0) {
             store_row<E, Tout>(xrot + p * D + lane * E, v1[0], true);
           } else {
-            pre_rotate_regs<Gm, 1, Tout>(v1, quads + static_cast<size_t>(e) * C::TAB_QUADS, xrot + p * D, buf, lane);
+            pre_rotate_regs<Gm, 1, Tout, C::TBUF_HALVES>(v1, quads + static_cast<size_t>(e) * C::TAB_QUADS, xrot + p * D, buf, lane);
           }
           shift_rows<G, E>(v);
         }
@@ -672,13 +737,16 @@ __device__ __forceinline__ void load_rows_l1(const Tz* zs0, float (&v)[G][Gm::E]
   }
 }
 
-template <class Gm, int G, typename Ts>
+template <class Gm, int G, typename Ts, bool HALVES = false>
 __device__ __forceinline__ void post_rotate_regs(float (&v)[G][Gm::E], const float4* tq, const RowMeta* m,
                                                  Ts* __restrict__ slot, float* buf, int lane) {
   constexpr int E = Gm::E;
   l1_fwd<Gm, G, 0>(v, tq, lane);
 #pragma unroll
-  for (int g = 0; g < G; ++g) to_layout2<E>(v[g], buf, lane);
+  for (int g = 0; g < G; ++g) {
+    if constexpr (HALVES) to_layout2_halves<E>(v[g], buf, lane);
+    else to_layout2<E>(v[g], buf, lane);
+  }
   l2_fwd<Gm, G, Gm::P>(v, tq, lane);
   // gate, round, and write each row with 16-byte stores: the row goes through
   // the warp's transpose buffer in natural order first
@@ -709,12 +777,12 @@ __device__ __forceinline__ void post_rotate_rows_smem(const Tz* zs0, const float
 // slot[r] = g_r * B(phi_e) z_p for bucket positions p (z already scaled by
 // alpha), r = rows[p], e = idx[r].
 template <int E, typename Tz, typename Ts>
-__global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS, StagedCfg<E, Tz>::MIN_BLOCKS) void post_rotate_fast_kernel(
+__global__ __launch_bounds__(StagedCfg<E, Tz, false>::THREADS, StagedCfg<E, Tz, false>::MIN_BLOCKS) void post_rotate_fast_kernel(
     const Tz* __restrict__ z, const int32_t* __restrict__ idx, const float* __restrict__ gates,
     const int32_t* __restrict__ rows, const float4* __restrict__ quads, long long R, int N, Ts* __restrict__ slot) {
   pdl_wait();
   pdl_trigger();
-  using C = StagedCfg<E, Tz>;
+  using C = StagedCfg<E, Tz, false>;
   using Gm = typename C::Gm;
   constexpr int G = C::G, D = Gm::D;
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -774,7 +842,7 @@ __global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS, StagedCfg<E, Tz>::MIN_BL
         RowMeta m[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, j * G + g);
-        post_rotate_regs<Gm, G, Ts>(v, quads + static_cast<size_t>(e0) * C::TAB_QUADS, m, slot, buf, lane);
+        post_rotate_regs<Gm, G, Ts, C::TBUF_HALVES>(v, quads + static_cast<size_t>(e0) * C::TAB_QUADS, m, slot, buf, lane);
       } else {
 #pragma unroll 1
         for (int g = 0; g < G; ++g) {
@@ -784,7 +852,7 @@ __global__ __launch_bounds__(StagedCfg<E, Tz>::THREADS, StagedCfg<E, Tz>::MIN_BL
             float v1[1][E];
 #pragma unroll
             for (int q = 0; q < E; ++q) v1[0][q] = v[0][q];
-            post_rotate_regs<Gm, 1, Ts>(v1, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS, m1, slot, buf,
+            post_rotate_regs<Gm, 1, Ts, C::TBUF_HALVES>(v1, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS, m1, slot, buf,
                                         lane);
           }
           shift_rows<G, E>(v);

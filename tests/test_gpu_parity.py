@@ -128,16 +128,31 @@ def test_large_workloads_sampled(name):
 
 # -- the boundary's maximum sizes ------------------------------------------------------
 
+def _compare_all_tokens_with_buckets(inp, gpu):
+    """Every token through the oracle's per-token expert (no dense experts,
+    for large d), plus the bucket arrays against the oracle's buckets."""
+    c, o, r = O.buckets(gpu["idx"], inp.wl.n_experts)
+    assert np.array_equal(gpu["counts"], c) and np.array_equal(gpu["offsets"], o)
+    assert np.array_equal(gpu["rows"], r)
+    compare(inp, gpu, tokens=np.arange(inp.wl.tokens))
+
+
+@pytest.mark.parametrize("N,T,dt", [(16, 70, "f32"), (64, 301, "bf16")])
+def test_forward_parity_d2048(N, T, dt):
+    """d = 2048: one row per warp, the pre-rotation switching layouts through
+    half a float32 row; several experts per warp range and a ragged tail."""
+    wl = W.custom("d2k", d=2048, n_experts=N, k=2, tokens=T, dtype=dt, bias_var=0.5,
+                  outlier_frac=0.005, outlier_scale=50.0)
+    inp = W.generate(wl, seed=N + T)
+    _compare_all_tokens_with_buckets(inp, run_cuda(inp))
+
+
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
 def test_maximum_d(dt):
     """d = 4096, the largest d the boundary accepts: 12 stages, one row per warp."""
     wl = W.custom("dmax", d=4096, n_experts=4, k=2, tokens=37, dtype=dt, bias_var=0.5)
     inp = W.generate(wl, seed=11)
-    gpu = run_cuda(inp)
-    c, o, r = O.buckets(gpu["idx"], wl.n_experts)
-    assert np.array_equal(gpu["counts"], c) and np.array_equal(gpu["offsets"], o)
-    assert np.array_equal(gpu["rows"], r)
-    compare(inp, gpu, tokens=np.arange(wl.tokens))
+    _compare_all_tokens_with_buckets(inp, run_cuda(inp))
 
 
 def test_maximum_experts_and_k():
