@@ -737,8 +737,13 @@ __device__ __forceinline__ void load_rows_l1(const Tz* zs0, float (&v)[G][Gm::E]
   }
 }
 
-template <class Gm, int G, typename Ts, bool HALVES = false>
-__device__ __forceinline__ void post_rotate_regs(float (&v)[G][Gm::E], const float4* tq, const RowMeta* m,
+// meta_of(g): row and gate of row g of the group.  At d <= 512 each row
+// leaves straight from layout 2 (a warp store covers 32 consecutive
+// elements: two whole sectors in bf16); from d = 1024 on it goes through the
+// transpose buffer in natural order and leaves as 16-byte stores, which
+// measured faster there.
+template <class Gm, int G, typename Ts, bool HALVES = false, class MetaOf>
+__device__ __forceinline__ void post_rotate_regs(float (&v)[G][Gm::E], const float4* tq, MetaOf meta_of,
                                                  Ts* __restrict__ slot, float* buf, int lane) {
   constexpr int E = Gm::E;
   l1_fwd<Gm, G, 0>(v, tq, lane);
@@ -748,30 +753,38 @@ __device__ __forceinline__ void post_rotate_regs(float (&v)[G][Gm::E], const flo
     else to_layout2<E>(v[g], buf, lane);
   }
   l2_fwd<Gm, G, Gm::P>(v, tq, lane);
-  // gate, round, and write each row with 16-byte stores: the row goes through
-  // the warp's transpose buffer in natural order first
-  constexpr int NCH = Gm::D * static_cast<int>(sizeof(Ts)) / 16;  // 16-byte chunks per row
-  Ts* row_buf = reinterpret_cast<Ts*>(buf);
+  if constexpr (E <= 16) {
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float gt = m[g].gate;
+    for (int g = 0; g < G; ++g) {
+      const RowMeta mg = meta_of(g);
+      Ts* dst = slot + static_cast<size_t>(mg.row) * Gm::D + lane;
 #pragma unroll
-    for (int q = 0; q < E; ++q) row_buf[q * 32 + lane] = from_f32<Ts>(gt * v[g][q]);
-    __syncwarp();
-    uint4* dst = reinterpret_cast<uint4*>(slot + static_cast<size_t>(m[g].row) * Gm::D);
-    const uint4* src = reinterpret_cast<const uint4*>(row_buf);
+      for (int q = 0; q < E; ++q) dst[q * 32] = from_f32<Ts>(mg.gate * v[g][q]);
+    }
+  } else {
+    constexpr int NCH = Gm::D * static_cast<int>(sizeof(Ts)) / 16;  // 16-byte chunks per row
+    Ts* row_buf = reinterpret_cast<Ts*>(buf);
 #pragma unroll
-    for (int c = lane; c < NCH; c += 32) dst[c] = src[c];
-    __syncwarp();
+    for (int g = 0; g < G; ++g) {
+      const RowMeta mg = meta_of(g);
+#pragma unroll
+      for (int q = 0; q < E; ++q) row_buf[q * 32 + lane] = from_f32<Ts>(mg.gate * v[g][q]);
+      __syncwarp();
+      uint4* dst = reinterpret_cast<uint4*>(slot + static_cast<size_t>(mg.row) * Gm::D);
+      const uint4* src = reinterpret_cast<const uint4*>(row_buf);
+#pragma unroll
+      for (int c = lane; c < NCH; c += 32) dst[c] = src[c];
+      __syncwarp();
+    }
   }
 }
 
-template <class Gm, int G, typename Tz, typename Ts>
-__device__ __forceinline__ void post_rotate_rows_smem(const Tz* zs0, const float4* tq, const RowMeta* m,
+template <class Gm, int G, typename Tz, typename Ts, class MetaOf>
+__device__ __forceinline__ void post_rotate_rows_smem(const Tz* zs0, const float4* tq, MetaOf meta_of,
                                                       Ts* __restrict__ slot, float* buf, int lane) {
   float v[G][Gm::E];
   load_rows_l1<Gm, G, Tz>(zs0, v, lane);
-  post_rotate_regs<Gm, G, Ts>(v, tq, m, slot, buf, lane);
+  post_rotate_regs<Gm, G, Ts>(v, tq, meta_of, slot, buf, lane);
 }
 
 // slot[r] = g_r * B(phi_e) z_p for bucket positions p (z already scaled by
@@ -839,10 +852,16 @@ __global__ __launch_bounds__(StagedCfg<E, Tz, false>::THREADS, StagedCfg<E, Tz, 
       load_rows_l1<Gm, G, Tz>(cur, v, lane);
       __syncwarp();  // all lanes have read the staged rows before buf (which aliases them) is written
       if (same == gm && p0 + G <= R) {
-        RowMeta m[G];
+        const float4* tq = quads + static_cast<size_t>(e0) * C::TAB_QUADS;
+        if constexpr (E <= 32) {  // metadata fetched at the store: fewer live registers
+          post_rotate_regs<Gm, G, Ts, C::TBUF_HALVES>(
+              v, tq, [&](int g) { return shfl_meta(mine, j * G + g); }, slot, buf, lane);
+        } else {
+          RowMeta m[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, j * G + g);
-        post_rotate_regs<Gm, G, Ts, C::TBUF_HALVES>(v, quads + static_cast<size_t>(e0) * C::TAB_QUADS, m, slot, buf, lane);
+          for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, j * G + g);
+          post_rotate_regs<Gm, G, Ts, C::TBUF_HALVES>(v, tq, [&](int g) { return m[g]; }, slot, buf, lane);
+        }
       } else {
 #pragma unroll 1
         for (int g = 0; g < G; ++g) {
@@ -852,19 +871,24 @@ __global__ __launch_bounds__(StagedCfg<E, Tz, false>::THREADS, StagedCfg<E, Tz, 
             float v1[1][E];
 #pragma unroll
             for (int q = 0; q < E; ++q) v1[0][q] = v[0][q];
-            post_rotate_regs<Gm, 1, Ts, C::TBUF_HALVES>(v1, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS, m1, slot, buf,
-                                        lane);
+            post_rotate_regs<Gm, 1, Ts, C::TBUF_HALVES>(v1, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS,
+                                                        [&](int) { return m1[0]; }, slot, buf, lane);
           }
           shift_rows<G, E>(v);
         }
       }
     } else {
       if (same == gm && p0 + G <= R) {
-        RowMeta m[G];
+        const float4* tq = quads + static_cast<size_t>(e0) * C::TAB_QUADS;
+        if constexpr (E <= 32) {  // metadata fetched at the store: fewer live registers
+          post_rotate_rows_smem<Gm, G, Tz, Ts>(cur, tq, [&](int g) { return shfl_meta(mine, j * G + g); }, slot, tbuf,
+                                               lane);
+        } else {
+          RowMeta m[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, j * G + g);
-        post_rotate_rows_smem<Gm, G, Tz, Ts>(cur, quads + static_cast<size_t>(e0) * C::TAB_QUADS, m, slot, tbuf,
-                                             lane);
+          for (int g = 0; g < G; ++g) m[g] = shfl_meta(mine, j * G + g);
+          post_rotate_rows_smem<Gm, G, Tz, Ts>(cur, tq, [&](int g) { return m[g]; }, slot, tbuf, lane);
+        }
       } else {
 #pragma unroll 1
         for (int g = 0; g < G; ++g) {
@@ -872,7 +896,7 @@ __global__ __launch_bounds__(StagedCfg<E, Tz, false>::THREADS, StagedCfg<E, Tz, 
           const RowMeta m1[1] = {shfl_meta(mine, j * G + g)};
           if (m1[0].ex < 0) continue;
           post_rotate_rows_smem<Gm, 1, Tz, Ts>(cur + g * D, quads + static_cast<size_t>(m1[0].ex) * C::TAB_QUADS,
-                                               m1, slot, tbuf, lane);
+                                               [&](int) { return m1[0]; }, slot, tbuf, lane);
         }
       }
     }
