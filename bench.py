@@ -367,7 +367,10 @@ def run_ours(args, wl):
             entry = {"launches": n, "total_ms": ms, "share": ms / max(1e-9, sum(v[1] for v in kt.values())),
                      "avg_us": 1e3 * ms / n}
             kernels[name] = entry
-        dom = max(kt.items(), key=lambda kv: kv[1][1])[0]
+        # the dominant kernel of the critical path: the table build runs on the
+        # side stream, overlapped with the router
+        main = {k: v for k, v in kt.items() if k not in SIDE_STREAM_KERNELS} or kt
+        dom = max(main.items(), key=lambda kv: kv[1][1])[0]
         roof = roofline_entry(dom, kt[dom], costs, peaks, clk, workload=wl.name)
         flops = 2.0 * T * wl.k * wl.d ** 2
         bytes_alg = algorithmic_bytes(wl)
@@ -417,6 +420,8 @@ def algorithmic_bytes(wl):
 
 
 # Launch names of the library -> kernel names in the ncu summaries.
+SIDE_STREAM_KERNELS = {"rot_table"}
+
 NCU_KERNEL = {"post_rotate": "post_rotate_fast_kernel", "pre_rotate": "pre_rotate_fast_kernel",
               "ternary_gemm_tc": "ternary_gemm_tc_kernel", "router_tc": "router_tc_kernel",
               "combine": "combine_kernel", "rot_table": "rot_quads_kernel"}
