@@ -621,7 +621,7 @@ int host_pipe(HostPipe** out) {
 struct HostPlan {
   int chunk, nchunks;
   int start[kHostMaxChunks + 1];  // chunk c = tokens start[c] .. start[c+1]-1
-  size_t x_dev, y_dev, idx, gates, counts, offsets, rows, moe, total;
+  size_t x_dev, y_dev, idx, gates, counts, offsets, rows, parts, moe, total;
 };
 
 // Chunks of `chunk` tokens; after the first chunk, the last chunk's worth is
@@ -660,6 +660,7 @@ HostPlan make_host_plan(int d, int N, int T, int k, int xdt, int chunk) {
   h.counts = take(static_cast<size_t>(N) * 4);
   h.offsets = take(static_cast<size_t>(N + 1) * 4);
   h.rows = take(rc * 4);
+  h.parts = take(static_cast<size_t>(3) * N * d * 2);  // W_g split once per call (tensor-core router)
   const Plan p = make_plan(d, N, h.chunk, k, xdt);
   h.moe = take(p.fwd_end + p.rt_end);
   h.total = off;
@@ -749,14 +750,41 @@ int bfmoe_unpack_base(const uint32_t* w_packed, int d, uint16_t* w_bf16, bfmoe_s
   return ok();
 }
 
+namespace {
+
+// The exact 3-way bf16 split of W_g ([3N][d]: hi, mid, lo parts per row block).
+cudaError_t split_gate_weights(const float* w_gate, int N, int d, __nv_bfloat16* parts, cudaStream_t s) {
+  const long long nw = static_cast<long long>(N) * d;
+  return launch("router_split", s, [&] { pdl_launch(router_split_kernel, grid_for(nw, 256, 2048), 256, 0, s, w_gate, nw, parts); });
+}
+
+bool tc_router_path(int x_dtype, int d) { return x_dtype == BFMOE_BF16 && d % kGemmBK == 0; }
+
+// Router + buckets; `parts_ready` (or null) is W_g already split by
+// split_gate_weights, which a caller routing several token chunks with the
+// same weights does once.
+int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_gate, const float* bias, int n_experts,
+                     int k, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, int32_t* rows, void* ws,
+                     size_t ws_bytes, cudaStream_t s, const __nv_bfloat16* parts_ready);
+
+}  // namespace
+
 int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_gate, const float* bias,
                       int n_experts, int k, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets,
                       int32_t* rows, void* ws, size_t ws_bytes, bfmoe_stream_t stream) {
+  return router_topk_impl(x, x_dtype, T, d, w_gate, bias, n_experts, k, idx, gates, counts, offsets, rows, ws,
+                          ws_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+namespace {
+
+int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_gate, const float* bias, int n_experts,
+                     int k, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, int32_t* rows, void* ws,
+                     size_t ws_bytes, cudaStream_t s, const __nv_bfloat16* parts_ready) {
   int rc = check_sizes(d, n_experts, T, k);
   if (rc) return rc;
   if ((rc = check_dtype(x_dtype))) return rc;
   if (!counts || !offsets) return fail(BFMOE_EINVAL, "router_topk: NULL counts/offsets");
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int N = n_experts;
   cudaError_t e;
   if (T == 0) {
@@ -773,14 +801,16 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
   int32_t* totals = reinterpret_cast<int32_t*>(W + p.totals);
   const long long R = static_cast<long long>(T) * k;
 
-  const bool tc_router = x_dtype == BFMOE_BF16 && d % kGemmBK == 0;
+  const bool tc_router = tc_router_path(x_dtype, d);
   if (tc_router) {
     // tensor cores: exact 3-way bf16 split of W_g, top-k fused in the epilogue
     if (!aligned16(x)) return fail(BFMOE_EINVAL, "router_topk: x must be 16-byte aligned");
-    __nv_bfloat16* parts = reinterpret_cast<__nv_bfloat16*>(W + p.wg_parts);
-    const long long nw = static_cast<long long>(N) * d;
-    e = launch("router_split", s, [&] { pdl_launch(router_split_kernel, grid_for(nw, 256, 2048), 256, 0, s, w_gate, nw, parts); });
-    if (e != cudaSuccess) return cuda_fail(e, "router_topk: split");
+    const __nv_bfloat16* parts = parts_ready;
+    if (!parts) {
+      __nv_bfloat16* own = reinterpret_cast<__nv_bfloat16*>(W + p.wg_parts);
+      if ((e = split_gate_weights(w_gate, N, d, own, s)) != cudaSuccess) return cuda_fail(e, "router_topk: split");
+      parts = own;
+    }
     const int BN = N >= 128 ? 128 : (N > 32 ? 64 : (N > 16 ? 32 : 16));
     CUtensorMap tx, tw;
     if (!make_tmap_bf16(&tx, x, d, T, kGemmBM) || !make_tmap_bf16(&tw, parts, d, 3LL * N, BN))
@@ -831,6 +861,8 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d, const float* w_g
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scatter");
   return ok();
 }
+
+}  // namespace
 
 int bfmoe_router_topk_noalloc(const void* x, int x_dtype, int T, int d, const float* w_gate, const float* bias,
                               int n_experts, int k, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets,
@@ -913,6 +945,12 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward_host: fork");
   rc = build_weight_tables(layer, bf16, pc, Wm, ss->stream);
   if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return cuda_fail(e, "moe_forward_host: join record");
+  // W_g is split once for all chunks, while the first chunk is copied in
+  __nv_bfloat16* parts = nullptr;
+  if (rc == BFMOE_OK && tc_router_path(x_dtype, d)) {
+    parts = reinterpret_cast<__nv_bfloat16*>(W + hp.parts);
+    if ((e = split_gate_weights(w_gate, N, d, parts, s)) != cudaSuccess) rc = cuda_fail(e, "moe_forward_host: split");
+  }
   for (int c = 0; c < hp.nchunks && rc == BFMOE_OK; ++c) {
     const int t0 = hp.start[c], Tc = hp.start[c + 1] - t0;
     const size_t o = static_cast<size_t>(t0) * row_bytes, n = static_cast<size_t>(Tc) * row_bytes;
@@ -922,8 +960,8 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
       rc = cuda_fail(e, "moe_forward_host: copy in");
       break;
     }
-    rc = bfmoe_router_topk(x_dev + o, x_dtype, Tc, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows,
-                           Wm + pc.fwd_end, pc.rt_end, stream);
+    rc = router_topk_impl(x_dev + o, x_dtype, Tc, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows,
+                          Wm + pc.fwd_end, pc.rt_end, s, parts);
     if (c == 0 && (e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) rc = cuda_fail(e, "moe_forward_host: join");
     if (rc) break;
     rc = forward_body(layer, x_dev + o, bf16, Tc, k, idx, gates, rows, y_dev + o, make_plan(d, N, Tc, k, x_dtype), Wm,
