@@ -194,9 +194,8 @@ size_t bfmoe_moe_workspace_size(int d, int n_experts, int T, int k, int x_dtype)
 /*
  * Router and expert forward from and to HOST memory, the host <-> device
  * copies overlapped with the work.  The T tokens are cut into chunks of
- * `chunk` tokens (chunk <= 0: about T/2, at least 2048; after a first chunk,
- * the last chunk's worth is cut into halves down to 512 tokens, so that the
- * unoverlapped work and copy of the last chunk are short); chunk i's copy in,
+ * `chunk` tokens, the last one taking the rest (chunk <= 0: six about equal
+ * chunks of at least 2048 tokens; at most 64 chunks); chunk i's copy in,
  * chunk i-1's router + forward and chunk i-2's copy out run at the same time
  * on a library-owned copy-in stream, `stream` and a library-owned copy-out
  * stream, ordered with events.  Each token's output is that of
@@ -210,8 +209,9 @@ size_t bfmoe_moe_workspace_size(int d, int n_experts, int T, int k, int x_dtype)
  *             stream before reading it)
  *   chunk     tokens per chunk, or <= 0 for the default
  *   ws        device scratch of bfmoe_moe_host_workspace_size(...) bytes (the
- *             device copies of x and y, one chunk's routing and one chunk's
- *             bfmoe_moe_forward scratch), 256-byte aligned
+ *             device copies of x and y, the split gate weights, one chunk's
+ *             routing and one chunk's bfmoe_moe_forward scratch), 256-byte
+ *             aligned
  * The copy streams and their events are created once per device on first use
  * (make that first call before any stream capture); after that the whole call
  * is stream-ordered and can be captured in a CUDA graph, copies included.

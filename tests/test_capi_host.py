@@ -82,8 +82,9 @@ def test_host_call_checks_before_any_launch(L):
 def test_host_workspace_size(L):
     bf = capi.BFMOE_BF16
     full = L.bfmoe_moe_host_workspace_size(512, 256, 16384, 2, bf, 0)
-    one = L.bfmoe_moe_workspace_size(512, 256, 8192, 2, bf)
-    # device x and y for all tokens plus one default chunk (T/2) of scratch
+    one = L.bfmoe_moe_workspace_size(512, 256, 2816, 2, bf)
+    # device x and y for all tokens plus one default chunk (T/6, rounded up
+    # to 128 tokens) of scratch
     assert full >= 2 * 16384 * 512 * 2 + one and full % 256 == 0
     assert L.bfmoe_moe_host_workspace_size(512, 256, 16384, 2, bf, 16384) > full  # one big chunk needs more
     assert L.bfmoe_moe_host_workspace_size(500, 256, 16384, 2, bf, 0) == 0
