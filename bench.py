@@ -373,7 +373,10 @@ def run_ours(args, wl):
         # side stream, overlapped with the router
         main = {k: v for k, v in kt.items() if k not in SIDE_STREAM_KERNELS} or kt
         dom = max(main.items(), key=lambda kv: kv[1][1])[0]
-        roof = roofline_entry(dom, kt[dom], costs, peaks, clk, workload=wl.name)
+        # a contraction timed inside a long step runs under the power cap:
+        # its peak is then the sustained GEMM figure, else the burst one
+        long_step = total_ms / args.steps > 1.0
+        roof = roofline_entry(dom, kt[dom], costs, peaks, clk, workload=wl.name, sustained=long_step)
         flops = 2.0 * T * wl.k * wl.d ** 2
         bytes_alg = algorithmic_bytes(wl)
         t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_alg / (peaks["hbm_gbs"] * 1e9))
@@ -468,14 +471,18 @@ def profiled_traffic(name, workload):
     return None
 
 
-def roofline_entry(name, kt_entry, costs, peaks, clk, workload=None):
+def roofline_entry(name, kt_entry, costs, peaks, clk, workload=None, sustained=False):
     n, ms = kt_entry
     avg_s = ms / n / 1e3
     bound, work, unit = costs.get(name, ("hbm", float("nan"), "GB/s"))
     if bound == "tensor":
         achieved = work / avg_s / 1e12
-        peak = peaks["bf16_tflops"]
-        src = "bf16_tflops (measured burst)"
+        if sustained and peaks.get("bf16_tflops_sustained"):
+            peak = peaks["bf16_tflops_sustained"]
+            src = "bf16_tflops_sustained (measured; the kernel runs inside a step of more than 1 ms)"
+        else:
+            peak = peaks["bf16_tflops"]
+            src = "bf16_tflops (measured burst)"
     elif bound == "alu":
         achieved = work / avg_s / 1e12
         mhz = peaks.get("sm_max_mhz", 1965.0)
