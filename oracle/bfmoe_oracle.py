@@ -35,7 +35,7 @@ force.
 from __future__ import annotations
 
 import math
-from typing import Optional, Sequence, Tuple
+from typing import Optional, Tuple
 
 import numpy as np
 
@@ -309,27 +309,3 @@ def rel_l2_per_token(y: np.ndarray, y_ref: np.ndarray) -> np.ndarray:
     num = np.linalg.norm(y - y_ref, axis=1)
     den = np.maximum(np.linalg.norm(y_ref, axis=1), 1e-30)
     return num / den
-
-
-def oracle_run(inputs, tokens: Optional[Sequence[int]] = None):
-    """Route and run the whole workload ``inputs`` (a ``workloads.Inputs``).
-
-    With ``tokens`` given, only those token ids are routed and evaluated (the
-    sampled mode used at full sizes).  Returns a dict of idx, gates,
-    near_tie, logits and y (and, in full mode, the buckets).
-    """
-    x = inputs.x_f64()
-    if tokens is not None:
-        tokens = np.asarray(tokens, dtype=np.int64)
-        x = x[tokens]
-    k = inputs.wl.k
-    idx, gates, near, logits = route(x, inputs.w_gate, inputs.bias, k)
-    out = {"idx": idx, "gates": gates, "near_tie": near, "logits": logits}
-    if tokens is None:
-        out["counts"], out["offsets"], out["rows"] = buckets(idx, inputs.wl.n_experts)
-        out["y"] = forward(x, inputs.w_base, inputs.alpha, inputs.theta,
-                           inputs.phi, idx, gates)
-    else:
-        out["y"] = forward_tokens(x, inputs.w_base, inputs.alpha, inputs.theta,
-                                  inputs.phi, idx, gates)
-    return out
