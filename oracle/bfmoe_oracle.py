@@ -309,3 +309,108 @@ def rel_l2_per_token(y: np.ndarray, y_ref: np.ndarray) -> np.ndarray:
     num = np.linalg.norm(y - y_ref, axis=1)
     den = np.maximum(np.linalg.norm(y_ref, axis=1), 1e-30)
     return num / den
+
+
+# ---------------------------------------------------------------------------
+# Backward pass (training the rotations with the ternary base)
+# ---------------------------------------------------------------------------
+#
+# The pages train the angles jointly with the quantised base (technical
+# summary, section 2.4; arXiv abstract on the signalfieldnotes article: the
+# rotations are learned with quantisation-aware training).  They give no
+# formula; the gradients below are the chain rule of the forward above, for
+# a loss L with dL/dy = gy.  The ternary base gets the straight-through
+# estimate: dL/dW_base as if W_base were a real matrix (the usual estimator
+# for a quantised weight; its use to update a latent full-precision base is
+# the trainer's business).  The top-k selection is piecewise constant, so the
+# router's gradient flows through the k selected logits only.
+
+def stage_derivative(d: int, s: int, angles_s: np.ndarray, r: int) -> np.ndarray:
+    """d S_s / d a_r: zero except the 2 x 2 block of rotation r,
+    [[-sin a, -cos a], [cos a, -sin a]]."""
+    h = 1 << s
+    a = float(np.asarray(angles_s, dtype=np.float64)[r])
+    D = np.zeros((d, d))
+    for i in range(d):
+        if i & h or rotation_index(i, s) != r:
+            continue
+        j = i + h
+        D[i, i] = -math.sin(a)
+        D[i, j] = -math.cos(a)
+        D[j, i] = math.cos(a)
+        D[j, j] = -math.sin(a)
+    return D
+
+
+def butterfly_angle_grad(angles: np.ndarray, inp: np.ndarray, gout: np.ndarray) -> np.ndarray:
+    """Sum over rows of <gout, (d B / d a_{s,r}) inp> for every angle, from
+    the dense factorisation B = S_{L-1} ... S_0:
+    d B / d a_{s,r} = (S_{L-1} ... S_{s+1}) (d S_s / d a_r) (S_{s-1} ... S_0).
+    ``inp`` and ``gout`` are [rows, d]; returns [L, d/2]."""
+    angles = np.asarray(angles, dtype=np.float64)
+    L, half = angles.shape
+    d = 2 * half
+    S = [stage_matrix(d, s, angles[s]) for s in range(L)]
+    out = np.zeros((L, half))
+    X = np.asarray(inp, dtype=np.float64)
+    G = np.asarray(gout, dtype=np.float64)
+    for s in range(L):
+        P = np.eye(d)
+        for q in range(s):
+            P = S[q] @ P
+        Q = np.eye(d)
+        for q in range(s + 1, L):
+            Q = S[q] @ Q
+        A = X @ P.T        # rows: stage-s inputs
+        Bg = G @ Q         # rows: Q^T gout, the gradient at stage-s outputs
+        for r in range(half):
+            Dr = stage_derivative(d, s, angles[s], r)
+            out[s, r] = np.einsum("ti,ij,tj->", Bg, Dr, A)
+    return out
+
+
+def backward(x, w_base, alpha, theta, phi, w_gate, bias, k, gy):
+    """Gradients of L with dL/dy = gy through the whole layer (router
+    included), with the routing of :func:`route`.  Returns a dict with dx,
+    dtheta, dphi (like theta), dw_base [d, d] (straight-through), dalpha,
+    dw_gate [N, d] and dbias [N] (None without a bias)."""
+    X = np.asarray(x, dtype=np.float64)
+    GY = np.asarray(gy, dtype=np.float64)
+    W = np.asarray(w_base, dtype=np.float64)
+    T, d = X.shape
+    N = np.asarray(w_gate).shape[0]
+    idx, g, _, _ = route(X, w_gate, bias, k)
+    dx = np.zeros_like(X)
+    dtheta = np.zeros(np.shape(theta))
+    dphi = np.zeros(np.shape(phi))
+    dW = np.zeros((d, d))
+    dalpha = 0.0
+    dg = np.zeros((T, k))
+    for e in np.unique(idx):
+        Bt = butterfly_matrix(theta[e])
+        Bp = butterfly_matrix(phi[e])
+        t, j = np.nonzero(idx == e)
+        U = X[t] @ Bt                     # rows u = B(theta)^T x
+        Z = float(alpha) * (U @ W.T)      # rows z = alpha W u
+        V = Z @ Bp.T                      # rows v = B(phi) z
+        dg[t, j] = np.einsum("ti,ti->t", V, GY[t])
+        dV = g[t, j][:, None] * GY[t]     # dL/dv
+        dZ = dV @ Bp                      # B(phi)^T dv
+        dU = float(alpha) * (dZ @ W)      # alpha W^T dz
+        dW += float(alpha) * (dZ.T @ U)
+        dalpha += float(np.einsum("ti,ti->", dZ, U @ W.T))
+        np.add.at(dx, t, dU @ Bt.T)       # B(theta) du
+        dphi[e] = butterfly_angle_grad(phi[e], Z, dV)
+        # u = B(theta)^T x: <du, dB^T/da x> = <dB/da du, x>
+        dtheta[e] = butterfly_angle_grad(theta[e], dU, X[t])
+    # router: g = softmax of the selected logits
+    dl = g * (dg - np.sum(g * dg, axis=1, keepdims=True))
+    dw_gate = np.zeros((N, d))
+    dbias = np.zeros(N)
+    for jj in range(k):
+        np.add.at(dw_gate, idx[:, jj], dl[:, jj][:, None] * X)
+        np.add.at(dbias, idx[:, jj], dl[:, jj])
+        dx += dl[:, jj][:, None] * np.asarray(w_gate, dtype=np.float64)[idx[:, jj]]
+    return {"dx": dx, "dtheta": dtheta, "dphi": dphi, "dw_base": dW, "dalpha": dalpha,
+            "dw_gate": dw_gate, "dbias": dbias if bias is not None else None,
+            "idx": idx, "gates": g}

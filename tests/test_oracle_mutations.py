@@ -116,3 +116,36 @@ def test_missing_bias_is_caught(monkeypatch):
     monkeypatch.setattr(O, "router_logits",
                         lambda x, W, b: np.asarray(x, float) @ np.asarray(W, float).T)
     assert _fails(pins.test_logits_include_bias)
+
+
+# -- backward pass: planted mistakes must fail the finite-difference pins ------
+
+def test_backward_wrong_rotation_derivative_is_caught(monkeypatch):
+    import tests.test_oracle_backward as bw
+    good = O.stage_derivative
+    monkeypatch.setattr(O, "stage_derivative", lambda d, s, a, r: good(d, s, a, r).T)
+    assert _fails(bw.test_backward_matches_finite_differences, 0, True, 2)
+
+
+def test_backward_untransposed_base_is_caught(monkeypatch):
+    import tests.test_oracle_backward as bw
+    good = O.backward
+
+    def bad(*a, **k):
+        g = good(*a, **k)
+        g["dw_base"] = g["dw_base"].T
+        return g
+    monkeypatch.setattr(O, "backward", bad)
+    assert _fails(bw.test_backward_matches_finite_differences, 0, True, 2)
+
+
+def test_backward_without_router_term_is_caught(monkeypatch):
+    import tests.test_oracle_backward as bw
+    good = O.backward
+
+    def bad(*a, **k):
+        g = good(*a, **k)
+        g["dw_gate"] = np.zeros_like(g["dw_gate"])
+        return g
+    monkeypatch.setattr(O, "backward", bad)
+    assert _fails(bw.test_backward_matches_finite_differences, 0, True, 2)
