@@ -325,47 +325,74 @@ def rel_l2_per_token(y: np.ndarray, y_ref: np.ndarray) -> np.ndarray:
 # the trainer's business).  The top-k selection is piecewise constant, so the
 # router's gradient flows through the k selected logits only.
 
+def rotation_derivative(a: float) -> np.ndarray:
+    """d/da of the Givens block [[cos a, -sin a], [sin a, cos a]]."""
+    return np.array([[-math.sin(a), -math.cos(a)], [math.cos(a), -math.sin(a)]])
+
+
 def stage_derivative(d: int, s: int, angles_s: np.ndarray, r: int) -> np.ndarray:
-    """d S_s / d a_r: zero except the 2 x 2 block of rotation r,
-    [[-sin a, -cos a], [cos a, -sin a]]."""
+    """d S_s / d a_r as a dense matrix: zero except the 2 x 2 block of
+    rotation r, :func:`rotation_derivative` of its angle."""
     h = 1 << s
     a = float(np.asarray(angles_s, dtype=np.float64)[r])
     D = np.zeros((d, d))
+    blk = rotation_derivative(a)
     for i in range(d):
         if i & h or rotation_index(i, s) != r:
             continue
         j = i + h
-        D[i, i] = -math.sin(a)
-        D[i, j] = -math.cos(a)
-        D[j, i] = math.cos(a)
-        D[j, j] = -math.sin(a)
+        D[np.ix_([i, j], [i, j])] = blk
     return D
+
+
+def stage_apply(angles_s: np.ndarray, X: np.ndarray, s: int, transpose: bool = False) -> np.ndarray:
+    """Rows of X times stage s (or its transpose): one step of
+    :func:`butterfly_apply`."""
+    d = X.shape[-1]
+    h = 1 << s
+    a = np.asarray(angles_s, dtype=np.float64)
+    lo = np.array([i for i in range(d) if not i & h])
+    hi = lo + h
+    r = np.array([rotation_index(int(i), s) for i in lo])
+    c, sn = np.cos(a[r]), np.sin(a[r])
+    if transpose:
+        sn = -sn
+    Y = np.array(X, dtype=np.float64, copy=True)
+    Y[..., lo] = c * X[..., lo] - sn * X[..., hi]
+    Y[..., hi] = sn * X[..., lo] + c * X[..., hi]
+    return Y
 
 
 def butterfly_angle_grad(angles: np.ndarray, inp: np.ndarray, gout: np.ndarray) -> np.ndarray:
     """Sum over rows of <gout, (d B / d a_{s,r}) inp> for every angle, from
-    the dense factorisation B = S_{L-1} ... S_0:
-    d B / d a_{s,r} = (S_{L-1} ... S_{s+1}) (d S_s / d a_r) (S_{s-1} ... S_0).
-    ``inp`` and ``gout`` are [rows, d]; returns [L, d/2]."""
+    the factorisation B = S_{L-1} ... S_0:
+    d B / d a_{s,r} = (S_{L-1} ... S_{s+1}) (d S_s / d a_r) (S_{s-1} ... S_0),
+    so the term is b^T (d S_s / d a_r) a with a = S_{s-1} ... S_0 inp (the
+    stage's input) and b = (S_{L-1} ... S_{s+1})^T gout; only the 2 x 2 block
+    of rotation r contributes.  ``inp`` and ``gout`` are [rows, d]; returns
+    [L, d/2]."""
     angles = np.asarray(angles, dtype=np.float64)
     L, half = angles.shape
     d = 2 * half
-    S = [stage_matrix(d, s, angles[s]) for s in range(L)]
-    out = np.zeros((L, half))
     X = np.asarray(inp, dtype=np.float64)
-    G = np.asarray(gout, dtype=np.float64)
-    for s in range(L):
-        P = np.eye(d)
-        for q in range(s):
-            P = S[q] @ P
-        Q = np.eye(d)
-        for q in range(s + 1, L):
-            Q = S[q] @ Q
-        A = X @ P.T        # rows: stage-s inputs
-        Bg = G @ Q         # rows: Q^T gout, the gradient at stage-s outputs
-        for r in range(half):
-            Dr = stage_derivative(d, s, angles[s], r)
-            out[s, r] = np.einsum("ti,ij,tj->", Bg, Dr, A)
+    ins = [X]
+    for s in range(L - 1):
+        ins.append(stage_apply(angles[s], ins[-1], s))
+    out = np.zeros((L, half))
+    Bg = np.asarray(gout, dtype=np.float64)
+    for s in range(L - 1, -1, -1):
+        A = ins[s]
+        h = 1 << s
+        for i in range(d):
+            if i & h:
+                continue
+            j = i + h
+            r = rotation_index(i, s)
+            D = rotation_derivative(angles[s][r])
+            pa = A[:, [i, j]]
+            pb = Bg[:, [i, j]]
+            out[s, r] = float(np.einsum("ti,ij,tj->", pb, D, pa))
+        Bg = stage_apply(angles[s], Bg, s, transpose=True)
     return out
 
 

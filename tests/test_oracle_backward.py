@@ -98,3 +98,37 @@ def test_zero_angles_reduce_to_a_scaled_dense_layer():
     gsum = gates.sum(axis=1)[:, None]
     dW = c["alpha"] * ((gsum * c["gy"]).T @ c["x"])
     assert np.allclose(g["dw_base"], dW, atol=1e-12)
+
+
+def test_stage_derivative_is_the_difference_quotient_of_the_stage():
+    rng = np.random.default_rng(8)
+    d = 8
+    for s in range(3):
+        ang = rng.uniform(-np.pi, np.pi, d // 2)
+        for r in range(d // 2):
+            p, m = ang.copy(), ang.copy()
+            p[r] += H
+            m[r] -= H
+            fd = (O.stage_matrix(d, s, p) - O.stage_matrix(d, s, m)) / (2 * H)
+            assert np.abs(O.stage_derivative(d, s, ang, r) - fd).max() < 1e-8
+
+
+def test_angle_gradient_equals_the_dense_factorisation():
+    # the stage-by-stage contraction against the dense prefix/suffix products
+    rng = np.random.default_rng(9)
+    d, L = 16, 4
+    ang = rng.uniform(-np.pi, np.pi, (L, d // 2))
+    X = rng.normal(size=(3, d))
+    G = rng.normal(size=(3, d))
+    S = [O.stage_matrix(d, s, ang[s]) for s in range(L)]
+    got = O.butterfly_angle_grad(ang, X, G)
+    for s in range(L):
+        P = np.eye(d)
+        for q in range(s):
+            P = S[q] @ P
+        Q = np.eye(d)
+        for q in range(s + 1, L):
+            Q = S[q] @ Q
+        for r in range(d // 2):
+            dB = Q @ O.stage_derivative(d, s, ang[s], r) @ P
+            assert abs(got[s, r] - np.einsum("ti,ij,tj->", G, dB, X)) < 1e-12

@@ -122,8 +122,8 @@ def test_missing_bias_is_caught(monkeypatch):
 
 def test_backward_wrong_rotation_derivative_is_caught(monkeypatch):
     import tests.test_oracle_backward as bw
-    good = O.stage_derivative
-    monkeypatch.setattr(O, "stage_derivative", lambda d, s, a, r: good(d, s, a, r).T)
+    good = O.rotation_derivative
+    monkeypatch.setattr(O, "rotation_derivative", lambda a: good(a).T)
     assert _fails(bw.test_backward_matches_finite_differences, 0, True, 2)
 
 
