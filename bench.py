@@ -143,6 +143,9 @@ def kernel_costs(wl, tables_bytes):
     return {
         # GEMM: 2 R d^2 flops on the tensor cores
         "ternary_gemm_tc": ("tensor", 2.0 * R * d * d, "TFLOP/s"),
+        # the whole expert in one kernel (pre-rotation, product, post-rotation,
+        # gate): its contraction is the 2 R d^2 of the product
+        "fused_expert": ("tensor", 2.0 * R * d * d, "TFLOP/s"),
         "ternary_gemm_simt": ("alu", 2.0 * R * d * d, "TFLOP/s"),
         # router product on the CUDA cores: 2 T N d flops
         "router_logits_simt": ("alu", 2.0 * T * N * d, "TFLOP/s"),
@@ -427,7 +430,7 @@ def algorithmic_bytes(wl):
 # Launch names of the library -> kernel names in the ncu summaries.
 SIDE_STREAM_KERNELS = {"rot_table"}
 
-NCU_KERNEL = {"post_rotate": "post_rotate_fast_kernel", "pre_rotate": "pre_rotate_fast_kernel",
+NCU_KERNEL = {"fused_expert": "fused_expert_kernel", "post_rotate": "post_rotate_fast_kernel", "pre_rotate": "pre_rotate_fast_kernel",
               "ternary_gemm_tc": "ternary_gemm_tc_kernel", "router_tc": "router_tc_kernel",
               "combine": "combine_kernel", "rot_table": "rot_quads_kernel"}
 

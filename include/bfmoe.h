@@ -72,6 +72,9 @@ typedef struct {
   float alpha;                /* scale of the ternary base                          */
   const float* theta;         /* [N][log2 d][d/2] input-side angles  (B(theta)^T)  */
   const float* phi;           /* [N][log2 d][d/2] output-side angles (B(phi))      */
+  const void* tables;         /* NULL, or this layer's weight tables written by
+                                 bfmoe_prepare_layer (then the calls read them
+                                 instead of rebuilding them per call)               */
 } bfmoe_layer;
 
 /*
@@ -129,8 +132,9 @@ int bfmoe_router_topk(const void* x, int x_dtype, int T, int d,
  * bfmoe_router_topk computes, using as scratch one fixed array inside the
  * library of BFMOE_NOALLOC_SCRATCH_BYTES (every GPU that loads the library
  * holds it until the process exits).  It allocates nothing.
- *   - Sizes whose scratch (bfmoe_workspace_size for these sizes) exceeds the
- *     array are rejected with BFMOE_EUNSUPPORTED before any launch.
+ *   - Sizes whose router scratch (bfmoe_router_scratch_size for these sizes)
+ *     exceeds the array are rejected with BFMOE_EUNSUPPORTED before any
+ *     launch.
  *   - The first call on a device looks up the array's device address with that
  *     device current; make that first call before any stream capture.
  *   - Every call shares the array: calls whose work overlaps on the GPU (on
@@ -188,6 +192,27 @@ int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int 
                       int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, int32_t* rows,
                       void* y, void* ws, size_t ws_bytes, bfmoe_stream_t stream);
 
+/*
+ * Build a layer's weight tables once (no counterpart on the pages, which store
+ * only the ternary base and the angles: technical summary, 2.2).  Every
+ * forward needs, besides the tokens, values that depend on the weights alone:
+ * cos and sin of every angle of theta and phi in the orders the rotation
+ * kernels read them, and the bf16 copy of the 2-bit base that the tensor cores
+ * multiply by.  Without prepared tables each forward call rebuilds them in its
+ * workspace; with `layer->tables` pointing at memory written by this call,
+ * bfmoe_forward, bfmoe_moe_forward and bfmoe_moe_forward_host read them
+ * instead (results identical bit for bit).  Rebuild after changing the
+ * layer's angles or base.
+ *   tables   device scratch of bfmoe_layer_tables_size(d, N) bytes, 256-byte
+ *            aligned, caller-owned (written; its contents are opaque)
+ * The layer's `tables` field is ignored by this call.  Returns BFMOE_EINVAL
+ * for a bad layer, BFMOE_EWORKSPACE for a short or misaligned buffer.
+ */
+int bfmoe_prepare_layer(const bfmoe_layer* layer, void* tables, size_t bytes, bfmoe_stream_t stream);
+
+/* Bytes of one layer's prepared weight tables (0 for invalid sizes). */
+size_t bfmoe_layer_tables_size(int d, int n_experts);
+
 /* Scratch bytes that bfmoe_moe_forward needs (0 for invalid sizes). */
 size_t bfmoe_moe_workspace_size(int d, int n_experts, int T, int k, int x_dtype);
 
@@ -227,6 +252,43 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
 size_t bfmoe_moe_host_workspace_size(int d, int n_experts, int T, int k, int x_dtype, int chunk);
 
 /*
+ * Backward pass of the layer (router included), for training the rotations
+ * jointly with the ternary base (technical summary, 2.4; the pages give no
+ * formula, so this is the chain rule of bfmoe_moe_forward's arithmetic).
+ * Given dL/dy, with the routing of the forward:
+ *   dg_r = <v_r, gy_t>, dv_r = g_r gy_t          (v_r = B(phi) alpha W u_r)
+ *   dphi_e  = sum over e's rows of d<dv, B(phi) z>/dphi,  dz = B(phi)^T dv
+ *   dw_base = alpha sum_r dz_r u_r^T   (straight-through: the gradient of W_base
+ *             taken as a real matrix, for the trainer's latent weights)
+ *   dalpha  = sum_r <dz_r, W_base u_r>,  du = alpha W_base^T dz
+ *   dtheta_e = sum over e's rows of d<du, B(theta)^T x>/dtheta,  dx += B(theta) du
+ *   router: dl_j = g_j (dg_j - sum_j' g_j' dg_j') for the k selected logits,
+ *   dw_gate[e] = sum dl x_t, dbias[e] = sum dl, dx_t += sum_j dl_j w_gate[e_j].
+ * Everything is computed in float32 on the CUDA cores (the forward's rows are
+ * recomputed in float32 from x; rotations are inverted stage by stage instead
+ * of storing their activations).  Angle gradients are summed with
+ * shared-memory atomics, so their last bits may differ between runs.
+ *   layer, x, x_dtype, T, k, w_gate: as for the forward (bias is not needed)
+ *   idx, gates, offsets, rows: the forward's routing (bfmoe_router_topk)
+ *   gy        device float [T][d]: dL/dy
+ *   dx        device float [T][d] (written)
+ *   dtheta, dphi  device float [N][log2 d][d/2] (written, zero for unused experts)
+ *   dw_base   device float [d][d] (written);  dalpha: device float [1] (written)
+ *   dw_gate   device float [N][d] (written);  dbias: device float [N] or NULL
+ *   ws        device scratch of bfmoe_backward_workspace_size(d, N, T, k)
+ *             bytes, 256-byte aligned
+ * Returns BFMOE_EINVAL / BFMOE_EWORKSPACE on bad arguments (nothing launched);
+ * routing indices out of range are reported through the device error word.
+ */
+int bfmoe_backward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, int k, const float* w_gate,
+                   const int32_t* idx, const float* gates, const int32_t* offsets, const int32_t* rows,
+                   const float* gy, float* dx, float* dtheta, float* dphi, float* dw_base, float* dalpha,
+                   float* dw_gate, float* dbias, void* ws, size_t ws_bytes, bfmoe_stream_t stream);
+
+/* Scratch bytes that bfmoe_backward needs (0 for invalid sizes). */
+size_t bfmoe_backward_workspace_size(int d, int n_experts, int T, int k);
+
+/*
  * Form expert e densely, alpha * B(phi_e) . W_base . B(theta_e)^T, in float32
  * (technical summary, 2.1).  For checking only.
  *   w_out     device float [d][d] (written), row = output
@@ -238,6 +300,14 @@ int bfmoe_materialize_expert(const bfmoe_layer* layer, int e, float* w_out,
  * sizes (one buffer serves both; calls on one stream may share it).
  * Returns 0 for invalid sizes. */
 size_t bfmoe_workspace_size(int d, int n_experts, int T, int k, int x_dtype);
+
+/* Scratch bytes that bfmoe_router_topk alone uses for these sizes (the part
+ * of bfmoe_workspace_size the router touches; it depends on the path taken:
+ * the CUDA-core router of float32 tokens, or of d not a multiple of 64, also
+ * keeps the float32 logits [T][N]).  bfmoe_router_topk_noalloc accepts the
+ * sizes for which this is at most BFMOE_NOALLOC_SCRATCH_BYTES.  Returns 0 for
+ * invalid sizes. */
+size_t bfmoe_router_scratch_size(int d, int n_experts, int T, int k, int x_dtype);
 
 /* Thread-local description of the last failed call ("" if none). */
 const char* bfmoe_last_error(void);

@@ -21,8 +21,9 @@ from .capi import BFMOE_BF16, BFMOE_F32, BfmoeError
 
 __all__ = [
     "BfmoeError", "Layer", "ButterflyMoE", "bfmoe_pack_base", "bfmoe_unpack_base", "bfmoe_router_topk",
-    "bfmoe_router_topk_noalloc", "bfmoe_moe_forward", "bfmoe_moe_workspace_size",
-    "bfmoe_forward", "bfmoe_materialize_expert", "bfmoe_workspace_size", "bfmoe_check_device_error",
+    "bfmoe_router_topk_noalloc", "bfmoe_moe_forward", "bfmoe_moe_workspace_size", "bfmoe_prepare_layer",
+    "bfmoe_layer_tables_size", "bfmoe_backward", "bfmoe_backward_workspace_size",
+    "bfmoe_forward", "bfmoe_materialize_expert", "bfmoe_workspace_size", "bfmoe_router_scratch_size", "bfmoe_check_device_error",
     "bfmoe_launch_count", "bfmoe_profile_enable", "bfmoe_profile_collect", "bfmoe_last_error", "workspace",
 ]
 
@@ -76,6 +77,11 @@ def bfmoe_launch_count() -> int:
 
 def bfmoe_workspace_size(d: int, n_experts: int, T: int, k: int, x_dtype: int) -> int:
     return int(capi.lib().bfmoe_workspace_size(d, n_experts, T, k, x_dtype))
+
+
+def bfmoe_router_scratch_size(d: int, n_experts: int, T: int, k: int, x_dtype: int) -> int:
+    """Scratch bytes the router alone uses (what bfmoe_router_topk_noalloc checks)."""
+    return int(capi.lib().bfmoe_router_scratch_size(d, n_experts, T, k, x_dtype))
 
 
 def workspace(d: int, n_experts: int, T: int, k: int, x_dtype: int, device=None):
@@ -176,7 +182,25 @@ class Layer:
         self.w_packed, self.theta, self.phi = w_packed, theta, phi
         self.alpha = float(alpha)
         self.c = capi.BfmoeLayer(self.d, self.n_experts, w_packed.data_ptr(), ctypes.c_float(alpha),
-                                 theta.data_ptr(), phi.data_ptr())
+                                 theta.data_ptr(), phi.data_ptr(), None)
+        self.tables = None
+
+    def prepare(self, stream=None):
+        """Build the weight tables once (bfmoe_prepare_layer); later calls with
+        this layer read them instead of rebuilding them per call."""
+        torch = _torch()
+        n = bfmoe_layer_tables_size(self.d, self.n_experts)
+        self.tables = torch.empty(max(n, 256), dtype=torch.uint8, device=self.theta.device)
+        self.c.tables = None
+        bfmoe_prepare_layer(self, self.tables, stream=stream)
+        self.c.tables = self.tables.data_ptr()
+        return self
+
+    def unprepare(self):
+        """Go back to building the tables per call."""
+        self.c.tables = None
+        self.tables = None
+        return self
 
     @classmethod
     def from_host(cls, w_base, alpha, theta, phi, device="cuda", stream=None):
@@ -187,6 +211,18 @@ class Layer:
         th = torch.as_tensor(theta, dtype=torch.float32).to(device).contiguous()
         ph = torch.as_tensor(phi, dtype=torch.float32).to(device).contiguous()
         return cls(packed, float(alpha), th, ph)
+
+
+def bfmoe_layer_tables_size(d: int, n_experts: int) -> int:
+    return int(capi.lib().bfmoe_layer_tables_size(d, n_experts))
+
+
+def bfmoe_prepare_layer(layer: "Layer", tables, stream=None):
+    """Write the layer's weight tables (cos/sin of the angles, bf16 base) into
+    ``tables`` (a device byte tensor of bfmoe_layer_tables_size bytes)."""
+    _need(tables, "tables")
+    capi.check(capi.lib().bfmoe_prepare_layer(ctypes.byref(layer.c), _ptr(tables), tables.numel(), _stream(stream)))
+    return tables
 
 
 def bfmoe_forward(layer: Layer, x, k: int, idx, gates, offsets, rows, ws, y=None, stream=None):
@@ -202,6 +238,40 @@ def bfmoe_forward(layer: Layer, x, k: int, idx, gates, offsets, rows, ws, y=None
         ctypes.byref(layer.c), _ptr(x), _dtype_code(x), T, k, _ptr(idx), _ptr(gates), _ptr(offsets),
         _ptr(rows), _ptr(y), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)))
     return y
+
+
+def bfmoe_backward_workspace_size(d: int, n_experts: int, T: int, k: int) -> int:
+    return int(capi.lib().bfmoe_backward_workspace_size(d, n_experts, T, k))
+
+
+def bfmoe_backward(layer: Layer, x, k: int, w_gate, routing, gy, bias_grad: bool = True, ws=None, stream=None):
+    """Gradients of the layer for dL/dy = gy (float32 [T][d]), with the
+    forward's routing (idx, gates, counts, offsets, rows).  Returns a dict of
+    float32 tensors dx, dtheta, dphi, dw_base, dalpha, dw_gate and dbias
+    (None when bias_grad is False)."""
+    torch = _torch()
+    _need(x, "x")
+    _need(w_gate, "w_gate", torch.float32)
+    _need(gy, "gy", torch.float32)
+    T, d = x.shape
+    if d != layer.d or tuple(gy.shape) != (T, d):
+        raise ValueError("x and gy must be [T][d] with the layer's d")
+    N = layer.n_experts
+    idx, gates, _counts, offsets, rows = routing
+    dev = x.device
+    if ws is None:
+        n = bfmoe_backward_workspace_size(d, N, T, k)
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+    f = dict(dtype=torch.float32, device=dev)
+    out = {"dx": torch.empty((T, d), **f), "dtheta": torch.empty_like(layer.theta),
+           "dphi": torch.empty_like(layer.phi), "dw_base": torch.empty((d, d), **f),
+           "dalpha": torch.empty((1,), **f), "dw_gate": torch.empty((N, d), **f),
+           "dbias": torch.empty((N,), **f) if bias_grad else None}
+    capi.check(capi.lib().bfmoe_backward(
+        ctypes.byref(layer.c), _ptr(x), _dtype_code(x), T, k, _ptr(w_gate), _ptr(idx), _ptr(gates), _ptr(offsets),
+        _ptr(rows), _ptr(gy), _ptr(out["dx"]), _ptr(out["dtheta"]), _ptr(out["dphi"]), _ptr(out["dw_base"]),
+        _ptr(out["dalpha"]), _ptr(out["dw_gate"]), _ptr(out["dbias"]), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
 
 
 def bfmoe_moe_workspace_size(d: int, n_experts: int, T: int, k: int, x_dtype: int) -> int:

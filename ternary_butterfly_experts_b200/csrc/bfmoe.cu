@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -12,8 +13,10 @@
 #include <string>
 #include <vector>
 
+#include "backward.cuh"
 #include "bucket.cuh"
 #include "common.cuh"
+#include "fused_tc.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "materialize.cuh"
@@ -160,17 +163,57 @@ int sm_count() {
 // ---------------------------------------------------------------------------
 // Workspace: router and forward share one buffer (stream-ordered).
 // ---------------------------------------------------------------------------
+// The weight-only tables of a layer: the cos/sin of theta and phi in the
+// layouts the rotation kernels read, and the bf16 copy of the base that the
+// tensor cores multiply by.  Built per call into the workspace, or once by
+// bfmoe_prepare_layer into caller memory.
+struct TabPlan {
+  size_t theta, phi, phi_pq, w_bf16, total;
+};
+
+TabPlan make_tab_plan(int d, int N) {
+  TabPlan t{};
+  const int L = ilog2(d);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  // quad layout for d >= 64, (c, s) pairs below; theta's table is followed
+  // directly by phi's (one launch writes both)
+  const size_t tab = d >= 64 ? static_cast<size_t>(N) * tab_quads(d / 32) * sizeof(float4)
+                             : static_cast<size_t>(N) * L * (d / 2) * sizeof(float2);
+  t.theta = take(2 * tab);
+  t.phi = t.theta + tab;
+  // pair quads of phi for the fused epilogue, [N][L][d/4]
+  t.phi_pq = take(d >= 64 ? static_cast<size_t>(N) * L * (d / 4) * sizeof(float4) : 0);
+  t.w_bf16 = take(d >= 64 ? static_cast<size_t>(d) * d * 2 : 0);
+  t.total = off;
+  return t;
+}
+
+// bf16 tokens with 64 <= d <= 512: the whole expert runs in one kernel
+// (fused_tc.cuh) and only the gated slots reach memory.
+bool fused_path(int xdt, int d) { return xdt == BFMOE_BF16 && d >= 64 && d <= 512; }
+
+// ---------------------------------------------------------------------------
+// Workspace: router and forward share one buffer (stream-ordered).
+// ---------------------------------------------------------------------------
 struct Plan {
   // forward
-  size_t tab_theta, tab_phi, w_bf16, xrot, z, slot, fwd_end;
+  size_t tabs, xrot, z, slot, fwd_end;
   // router
-  size_t logits, chunk_counts, totals, wg_parts, rt_end;
+  size_t logits, chunk_counts, totals, wg_parts, unsure, rt_end;
   size_t total;
 };
 
+// The router runs on the tensor cores for bf16 tokens whose width is a whole
+// number of 64-column k-blocks, else on the CUDA cores.
+bool tc_router_path(int x_dtype, int d) { return x_dtype == BFMOE_BF16 && d % kGemmBK == 0; }
+
 Plan make_plan(int d, int N, long long T, int k, int xdt) {
   Plan p{};
-  const int L = ilog2(d);
   const long long R = T * k;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -178,24 +221,25 @@ Plan make_plan(int d, int N, long long T, int k, int xdt) {
     off += align_up(bytes, 256);
     return o;
   };
-  // cos/sin tables: theta then phi (quad layout for d >= 64, (c, s) pairs below)
-  const size_t tab = d >= 64 ? static_cast<size_t>(N) * tab_quads(d / 32) * sizeof(float4)
-                             : static_cast<size_t>(N) * L * (d / 2) * sizeof(float2);
-  p.tab_theta = take(2 * tab);
-  p.tab_phi = p.tab_theta + tab;
-  p.w_bf16 = take(static_cast<size_t>(d) * d * 2);
-  p.xrot = take(static_cast<size_t>(R) * d * (xdt == BFMOE_BF16 ? 2 : 4));
-  // the bf16 tensor-core path keeps Z and the per-slot outputs in bf16
+  p.tabs = take(make_tab_plan(d, N).total);
+  // the bf16 tensor-core path keeps Z and the per-slot outputs in bf16; the
+  // fused path writes only the slots
   const size_t inter = (xdt == BFMOE_BF16 && d >= 64) ? 2 : 4;
-  p.z = take(static_cast<size_t>(R) * d * inter);
+  if (!fused_path(xdt, d)) {
+    p.xrot = take(static_cast<size_t>(R) * d * (xdt == BFMOE_BF16 ? 2 : 4));
+    p.z = take(static_cast<size_t>(R) * d * inter);
+  }
   p.slot = take(static_cast<size_t>(R) * d * inter);
   p.fwd_end = off;
   off = 0;
   const long long nchunks = (R + bucket_chunk(k) - 1) / bucket_chunk(k);
+  // float32 logits [T][N] (both routers keep them for the fix-up)
   p.logits = take(static_cast<size_t>(T) * N * 4);
   p.chunk_counts = take(static_cast<size_t>(std::max(1LL, nchunks)) * N * 4);
   p.totals = take(static_cast<size_t>(N) * 4);
   p.wg_parts = take(static_cast<size_t>(3) * N * d * 2);
+  // tokens whose float32 shortlist needs the float64 scan: count, spare, ids
+  p.unsure = take((2 + static_cast<size_t>(T)) * 4);
   p.rt_end = off;
   p.total = std::max(p.fwd_end, p.rt_end);
   return p;
@@ -404,7 +448,8 @@ cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const C
 
 template <int BN, int STAGES, int K>
 cudaError_t launch_router_tc_k(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
-                               int32_t* idx, float* gates, int32_t* cc, cudaStream_t s) {
+                               float eps_c, float* logits, int* unsure, int32_t* idx, float* gates,
+                               int32_t* cc, cudaStream_t s) {
   using Cfg = RouterTcCfg<BN, STAGES>;
   static std::atomic<uint64_t> done{0};
   if (needs_attr(done)) {
@@ -415,23 +460,24 @@ cudaError_t launch_router_tc_k(const CUtensorMap& tx, const CUtensorMap& tw, con
   }
   const int grid = (T + kGemmBM - 1) / kGemmBM;
   return launch("router_tc", s, [&] {
-    pdl_launch(router_tc_kernel<BN, STAGES, K>, grid, kRouterThreads, Cfg::SMEM_BYTES, s, tx, tw, bias, T, d, N, idx,
-               gates, cc);
+    pdl_launch(router_tc_kernel<BN, STAGES, K>, grid, kRouterThreads, Cfg::SMEM_BYTES, s, tx, tw, bias, T, d, N,
+               eps_c, logits, unsure, idx, gates, cc);
   });
 }
 
 template <int BN, int STAGES>
 cudaError_t launch_router_tc(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
-                             int k, int32_t* idx, float* gates, int32_t* cc, cudaStream_t s) {
+                             int k, float eps_c, float* logits, int* unsure, int32_t* idx, float* gates,
+                             int32_t* cc, cudaStream_t s) {
   switch (k) {
-    case 1: return launch_router_tc_k<BN, STAGES, 1>(tx, tw, bias, T, d, N, idx, gates, cc, s);
-    case 2: return launch_router_tc_k<BN, STAGES, 2>(tx, tw, bias, T, d, N, idx, gates, cc, s);
-    case 3: return launch_router_tc_k<BN, STAGES, 3>(tx, tw, bias, T, d, N, idx, gates, cc, s);
-    case 4: return launch_router_tc_k<BN, STAGES, 4>(tx, tw, bias, T, d, N, idx, gates, cc, s);
-    case 5: return launch_router_tc_k<BN, STAGES, 5>(tx, tw, bias, T, d, N, idx, gates, cc, s);
-    case 6: return launch_router_tc_k<BN, STAGES, 6>(tx, tw, bias, T, d, N, idx, gates, cc, s);
-    case 7: return launch_router_tc_k<BN, STAGES, 7>(tx, tw, bias, T, d, N, idx, gates, cc, s);
-    default: return launch_router_tc_k<BN, STAGES, 8>(tx, tw, bias, T, d, N, idx, gates, cc, s);
+    case 1: return launch_router_tc_k<BN, STAGES, 1>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
+    case 2: return launch_router_tc_k<BN, STAGES, 2>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
+    case 3: return launch_router_tc_k<BN, STAGES, 3>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
+    case 4: return launch_router_tc_k<BN, STAGES, 4>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
+    case 5: return launch_router_tc_k<BN, STAGES, 5>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
+    case 6: return launch_router_tc_k<BN, STAGES, 6>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
+    case 7: return launch_router_tc_k<BN, STAGES, 7>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
+    default: return launch_router_tc_k<BN, STAGES, 8>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
   }
 }
 
@@ -452,21 +498,23 @@ int check_forward_args(const bfmoe_layer* layer, const void* x, int x_dtype, int
   return BFMOE_OK;
 }
 
-// The inputs of the forward that depend on the weights only: the cos/sin
-// tables of theta and phi and, on the bf16 path, the bf16 copy of the base.
-int build_weight_tables(const bfmoe_layer* layer, bool bf16, const Plan& p, uint8_t* W, cudaStream_t s) {
+// The inputs of the forward that depend on the weights only (TabPlan), into
+// `tabs`: the cos/sin tables of theta and phi and, from d = 64 on, phi's pair
+// quads and the bf16 copy of the base for the tensor cores.
+int build_weight_tables(const bfmoe_layer* layer, uint8_t* tabs, cudaStream_t s) {
   const int d = layer->d, N = layer->n_experts, L = ilog2(d);
-  float2* tab_t = reinterpret_cast<float2*>(W + p.tab_theta);
-  float2* tab_p = reinterpret_cast<float2*>(W + p.tab_phi);
-  uint16_t* wbf = reinterpret_cast<uint16_t*>(W + p.w_bf16);
+  const TabPlan tp = make_tab_plan(d, N);
+  float2* tab_t = reinterpret_cast<float2*>(tabs + tp.theta);
+  float2* tab_p = reinterpret_cast<float2*>(tabs + tp.phi);
+  uint16_t* wbf = reinterpret_cast<uint16_t*>(tabs + tp.w_bf16);
   const long long nang = static_cast<long long>(N) * L * (d / 2);
   cudaError_t e;
   if (d >= 64) {
-    // one launch builds both tables (the phi table follows the theta table)
-    // and, on the bf16 path, the bf16 copy of the base for the tensor cores
+    // one launch builds both quad tables (the phi table follows the theta
+    // table) and the bf16 copy of the base
     const TabLayout tl = make_tab_layout(d / 32, L);
     const int tab_blocks = 2 * N;
-    const int exp_blocks = bf16 ? grid_for(static_cast<long long>(d) * (d / 16), 256, 1024) : 0;
+    const int exp_blocks = grid_for(static_cast<long long>(d) * (d / 16), 256, 1024);
     const size_t tab_smem = static_cast<size_t>(L) * d * sizeof(float);  // cos and sin of one expert
     static std::atomic<uint64_t> done{0};
     if (needs_attr(done)) {
@@ -476,9 +524,13 @@ int build_weight_tables(const bfmoe_layer* layer, bool bf16, const Plan& p, uint
     }
     e = launch("rot_table", s, [&] {
       rot_quads_kernel<<<tab_blocks + exp_blocks, 256, tab_smem, s>>>(
-          layer->theta, layer->phi, N, d, L, tl, reinterpret_cast<float4*>(tab_t), layer->w_packed,
-          bf16 ? wbf : nullptr);
+          layer->theta, layer->phi, N, d, L, tl, reinterpret_cast<float4*>(tab_t), layer->w_packed, wbf);
     });
+    if (e == cudaSuccess)
+      e = launch("rot_table", s, [&] {
+        rot_pairq_kernel<<<grid_for(nang / 2, 256, 4096), 256, 0, s>>>(
+            layer->phi, nang / 2, reinterpret_cast<float4*>(tabs + tp.phi_pq));
+      });
   } else {
     e = launch("rot_table", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->theta, nang, tab_t); });
     if (e == cudaSuccess)
@@ -488,21 +540,80 @@ int build_weight_tables(const bfmoe_layer* layer, bool bf16, const Plan& p, uint
   return BFMOE_OK;
 }
 
-// Pre-rotation, ternary product, post-rotation with gates, combine.
+template <int D>
+cudaError_t launch_fused(const CUtensorMap& tb, const __nv_bfloat16* x, const int32_t* idx, const float* gates,
+                         const int32_t* rows, const float4* tq, const float4* pq, long long R, int k, int N,
+                         float alpha, __nv_bfloat16* slot, cudaStream_t s) {
+  using C = FusedCfg<D>;
+  static std::atomic<uint64_t> done{0};
+  if (needs_attr(done)) {
+    cudaError_t e = cudaFuncSetAttribute(fused_expert_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set(done);
+  }
+  const long long tiles = (R + kGemmBM - 1) / kGemmBM;
+  const int grid = static_cast<int>(std::min<long long>(tiles, sm_count()));
+  return launch("fused_expert", s, [&] {
+    pdl_launch(fused_expert_kernel<D>, grid, kFusedThreads, C::SMEM_BYTES, s, tb, x, idx, gates, rows, tq, pq, R, k,
+               N, alpha, slot);
+  });
+}
+
+// Gated combine of the slots: y_t = sum_j slot[t k + j], one rounding.
+cudaError_t launch_combine(bool bf16, bool fast, const void* slot, int T, int k, int d, void* y, cudaStream_t s) {
+  const long long nv = static_cast<long long>(T) * (d / ((bf16 && fast) ? 8 : 4));
+  return launch("combine", s, [&] {
+    const int g = grid_for(nv, 256, sm_count() * 16);
+    if (bf16 && fast)
+      pdl_launch(combine_kernel<__nv_bfloat16, __nv_bfloat16>, g, 256, 0, s,
+                 static_cast<const __nv_bfloat16*>(slot), static_cast<long long>(T), k, d,
+                 static_cast<__nv_bfloat16*>(y));
+    else if (bf16)
+      combine_kernel<float, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d,
+                                                             static_cast<__nv_bfloat16*>(y));
+    else
+      combine_kernel<float, float><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d, static_cast<float*>(y));
+  });
+}
+
+// Pre-rotation, ternary product, post-rotation with gates, combine.  `tabs`
+// holds the weight tables (TabPlan), built per call or prepared once.
 int forward_body(const bfmoe_layer* layer, const void* x, bool bf16, int T, int k, const int32_t* idx,
-                 const float* gates, const int32_t* rows, void* y, const Plan& p, uint8_t* W, cudaStream_t s) {
+                 const float* gates, const int32_t* rows, void* y, const Plan& p, uint8_t* W, const uint8_t* tabs,
+                 cudaStream_t s) {
   const int d = layer->d, N = layer->n_experts, L = ilog2(d);
-  float2* tab_t = reinterpret_cast<float2*>(W + p.tab_theta);
-  float2* tab_p = reinterpret_cast<float2*>(W + p.tab_phi);
-  uint16_t* wbf = reinterpret_cast<uint16_t*>(W + p.w_bf16);
-  void* xrot = W + p.xrot;
-  void* z = W + p.z;
+  const TabPlan tp = make_tab_plan(d, N);
+  const float2* tab_t = reinterpret_cast<const float2*>(tabs + tp.theta);
+  const float2* tab_p = reinterpret_cast<const float2*>(tabs + tp.phi);
+  const uint16_t* wbf = reinterpret_cast<const uint16_t*>(tabs + tp.w_bf16);
   void* slot = W + p.slot;
   const long long R = static_cast<long long>(T) * k;
   const int wpr = words_per_row(d);
   const bool fast = d >= 64;
   cudaError_t e;
 
+  if (fused_path(bf16 ? BFMOE_BF16 : BFMOE_F32, d)) {
+    CUtensorMap tb;
+    if (!make_tmap_bf16(&tb, wbf, d, d, std::min(d, 256))) return fail(BFMOE_ECUDA, "forward: tensor map encoding failed");
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    const auto* tq = reinterpret_cast<const float4*>(tab_t);
+    const auto* pq = reinterpret_cast<const float4*>(tabs + tp.phi_pq);
+    auto* sb = static_cast<__nv_bfloat16*>(slot);
+    switch (d) {
+      case 64: e = launch_fused<64>(tb, xb, idx, gates, rows, tq, pq, R, k, N, layer->alpha, sb, s); break;
+      case 128: e = launch_fused<128>(tb, xb, idx, gates, rows, tq, pq, R, k, N, layer->alpha, sb, s); break;
+      case 256: e = launch_fused<256>(tb, xb, idx, gates, rows, tq, pq, R, k, N, layer->alpha, sb, s); break;
+      default: e = launch_fused<512>(tb, xb, idx, gates, rows, tq, pq, R, k, N, layer->alpha, sb, s); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "forward: fused expert kernel");
+    e = launch_combine(true, true, slot, T, k, d, y, s);
+    if (e != cudaSuccess) return cuda_fail(e, "forward: combine");
+    return ok();
+  }
+
+  void* xrot = W + p.xrot;
+  void* z = W + p.z;
   RotArgs ra{x, bf16, idx, gates, rows, tab_t, R, k, d, L, N, xrot, nullptr, s};
   e = fast ? dispatch_fast<PreRotateFast>(d, ra) : dispatch_e<PreRotate>(d, ra);
   if (e != cudaSuccess) return cuda_fail(e, "forward: pre-rotation");
@@ -539,19 +650,7 @@ int forward_body(const bfmoe_layer* layer, const void* x, bool bf16, int T, int 
   e = fast ? dispatch_fast<PostRotateFast>(d, rb) : dispatch_e<PostRotate>(d, rb);
   if (e != cudaSuccess) return cuda_fail(e, "forward: post-rotation");
 
-  const long long nv = static_cast<long long>(T) * (d / ((bf16 && fast) ? 8 : 4));
-  e = launch("combine", s, [&] {
-    const int g = grid_for(nv, 256, sm_count() * 16);
-    if (bf16 && fast)
-      pdl_launch(combine_kernel<__nv_bfloat16, __nv_bfloat16>, g, 256, 0, s,
-                 static_cast<const __nv_bfloat16*>(slot), static_cast<long long>(T), k, d,
-                 static_cast<__nv_bfloat16*>(y));
-    else if (bf16)
-      combine_kernel<float, __nv_bfloat16><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d,
-                                                             static_cast<__nv_bfloat16*>(y));
-    else
-      combine_kernel<float, float><<<g, 256, 0, s>>>(static_cast<const float*>(slot), T, k, d, static_cast<float*>(y));
-  });
+  e = launch_combine(bf16, fast, slot, T, k, d, y, s);
   if (e != cudaSuccess) return cuda_fail(e, "forward: combine");
   return ok();
 }
@@ -703,6 +802,106 @@ int noalloc_scratch(void** out) {
 
 }  // namespace
 
+namespace {
+
+// Workspace of bfmoe_backward.
+struct BwPlan {
+  size_t tab_t, tab_p, wt, U, Z, dU, dg, dl, part, dapart, total;
+  int slices, ra_blocks;
+};
+
+BwPlan make_bw_plan(int d, int N, long long T, int k) {
+  BwPlan b{};
+  const int L = ilog2(d);
+  const long long R = T * k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  const size_t tab = static_cast<size_t>(N) * L * (d / 2) * sizeof(float2);
+  b.tab_t = take(tab);
+  b.tab_p = take(tab);
+  b.wt = take(static_cast<size_t>(d) * words_per_row(d) * 4);
+  b.U = take(static_cast<size_t>(R) * d * 4);
+  b.Z = take(static_cast<size_t>(R) * d * 4);  // Z, then dZ in place, then the per-row dx
+  b.dU = take(static_cast<size_t>(R) * d * 4);
+  b.dg = take(static_cast<size_t>(R) * 4);
+  b.dl = take(static_cast<size_t>(R) * 4);
+  // the outer product dZ^T U in slices of the rows, at most 64 MB of partials
+  long long sl = (R + 2047) / 2048;
+  const long long cap = std::max(1LL, (64LL << 20) / (static_cast<long long>(d) * d * 4));
+  sl = std::max(1LL, std::min({sl, 16LL, cap}));
+  b.slices = static_cast<int>(sl);
+  b.part = take(static_cast<size_t>(sl) * d * d * 4);
+  b.ra_blocks = grid_for(static_cast<long long>(d) * d, 256, 1024);
+  b.dapart = take(static_cast<size_t>(b.ra_blocks) * 4);
+  b.total = off;
+  return b;
+}
+
+template <int E>
+struct BwRows {
+  static cudaError_t run(const void* x, bool bf16, const int32_t* idx, const int32_t* rows, const int32_t* offsets,
+                         const float* gates, const float* gy, const float2* tab_t, const float2* tab_p, long long R,
+                         int k, int d, int L, int N, float* U, float* Z, float* dU, float* dg, float* dtheta,
+                         float* dphi, int stage, cudaStream_t s) {
+    const size_t smem = static_cast<size_t>(L) * (d / 2) * sizeof(float);
+    static std::atomic<uint64_t> done{0};
+    if (needs_attr(done)) {
+      cudaFuncSetAttribute(bw_post_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, 12 * BFMOE_MAX_D * 2);
+      cudaFuncSetAttribute(bw_pre_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, 12 * BFMOE_MAX_D * 2);
+      attr_set(done);
+    }
+    if (stage == 0) {  // u = B(theta)^T x, bucket order, float32
+      const int grid = grid_for(R, 8, sm_count() * 16);
+      return launch("bw_pre_rotate", s, [&] {
+        if (bf16)
+          pre_rotate_kernel<E, __nv_bfloat16, float><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), idx,
+                                                                          rows, tab_t, R, k, d, L, N, U);
+        else
+          pre_rotate_kernel<E, float, float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), idx, rows, tab_t, R,
+                                                                  k, d, L, N, U);
+      });
+    }
+    if (stage == 1)
+      return launch("bw_post", s, [&] {
+        bw_post_kernel<E><<<N, 256, smem, s>>>(Z, gy, rows, offsets, gates, tab_p, d, L, k, N, R, Z, dg, dphi);
+      });
+    return launch("bw_pre", s, [&] {
+      bw_pre_kernel<E><<<N, 256, smem, s>>>(U, dU, rows, offsets, tab_t, d, L, R, Z, dtheta);
+    });
+  }
+};
+
+template <int E, typename... A>
+cudaError_t bw_rows(int d, A&&... a) {
+  (void)d;
+  return BwRows<E>::run(std::forward<A>(a)...);
+}
+
+cudaError_t bw_rows_dispatch(int d, const void* x, bool bf16, const int32_t* idx, const int32_t* rows,
+                             const int32_t* offsets, const float* gates, const float* gy, const float2* tab_t,
+                             const float2* tab_p, long long R, int k, int L, int N, float* U, float* Z, float* dU,
+                             float* dg, float* dtheta, float* dphi, int stage, cudaStream_t s) {
+#define BW_ARGS x, bf16, idx, rows, offsets, gates, gy, tab_t, tab_p, R, k, d, L, N, U, Z, dU, dg, dtheta, dphi, stage, s
+  switch (d) {
+    case 4: case 8: case 16: case 32: return BwRows<1>::run(BW_ARGS);
+    case 64: return BwRows<2>::run(BW_ARGS);
+    case 128: return BwRows<4>::run(BW_ARGS);
+    case 256: return BwRows<8>::run(BW_ARGS);
+    case 512: return BwRows<16>::run(BW_ARGS);
+    case 1024: return BwRows<32>::run(BW_ARGS);
+    case 2048: return BwRows<64>::run(BW_ARGS);
+    case 4096: return BwRows<128>::run(BW_ARGS);
+    default: return cudaErrorInvalidValue;
+  }
+#undef BW_ARGS
+}
+
+}  // namespace
+
 // ===========================================================================
 // C ABI
 // ===========================================================================
@@ -715,6 +914,11 @@ unsigned long long bfmoe_launch_count(void) { return g_launches.load(); }
 size_t bfmoe_workspace_size(int d, int n_experts, int T, int k, int x_dtype) {
   if (check_sizes(d, n_experts, T, k) != BFMOE_OK || check_dtype(x_dtype) != BFMOE_OK) return 0;
   return make_plan(d, n_experts, T, k, x_dtype).total;
+}
+
+size_t bfmoe_router_scratch_size(int d, int n_experts, int T, int k, int x_dtype) {
+  if (check_sizes(d, n_experts, T, k) != BFMOE_OK || check_dtype(x_dtype) != BFMOE_OK) return 0;
+  return make_plan(d, n_experts, T, k, x_dtype).rt_end;
 }
 
 int bfmoe_pack_base(const int8_t* w, int d, uint32_t* w_packed, bfmoe_stream_t stream) {
@@ -758,8 +962,6 @@ cudaError_t split_gate_weights(const float* w_gate, int N, int d, __nv_bfloat16*
   return launch("router_split", s, [&] { pdl_launch(router_split_kernel, grid_for(nw, 256, 2048), 256, 0, s, w_gate, nw, parts); });
 }
 
-bool tc_router_path(int x_dtype, int d) { return x_dtype == BFMOE_BF16 && d % kGemmBK == 0; }
-
 // Router + buckets; `parts_ready` (or null) is W_g already split by
 // split_gate_weights, which a caller routing several token chunks with the
 // same weights does once.
@@ -799,7 +1001,11 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
   float* logits = reinterpret_cast<float*>(W + p.logits);
   int32_t* cc = reinterpret_cast<int32_t*>(W + p.chunk_counts);
   int32_t* totals = reinterpret_cast<int32_t*>(W + p.totals);
+  int* unsure = reinterpret_cast<int*>(W + p.unsure);
   const long long R = static_cast<long long>(T) * k;
+  // the float32 error band that leaves a top-k undecided (router.cuh)
+  const float eps_c = 2e-5f * std::sqrt(static_cast<float>(d) / 2048.f);
+  if ((e = cudaMemsetAsync(unsure, 0, 8, s)) != cudaSuccess) return cuda_fail(e, "router_topk: memset");
 
   const bool tc_router = tc_router_path(x_dtype, d);
   if (tc_router) {
@@ -816,10 +1022,10 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
     if (!make_tmap_bf16(&tx, x, d, T, kGemmBM) || !make_tmap_bf16(&tw, parts, d, 3LL * N, BN))
       return fail(BFMOE_ECUDA, "router_topk: tensor map encoding failed");
     switch (BN) {
-      case 16: e = launch_router_tc<16, 4>(tx, tw, bias, T, d, N, k, idx, gates, cc, s); break;
-      case 32: e = launch_router_tc<32, 4>(tx, tw, bias, T, d, N, k, idx, gates, cc, s); break;
-      case 64: e = launch_router_tc<64, 4>(tx, tw, bias, T, d, N, k, idx, gates, cc, s); break;
-      default: e = launch_router_tc<128, 3>(tx, tw, bias, T, d, N, k, idx, gates, cc, s); break;
+      case 16: e = launch_router_tc<16, 4>(tx, tw, bias, T, d, N, k, eps_c, logits, unsure, idx, gates, cc, s); break;
+      case 32: e = launch_router_tc<32, 4>(tx, tw, bias, T, d, N, k, eps_c, logits, unsure, idx, gates, cc, s); break;
+      case 64: e = launch_router_tc<64, 4>(tx, tw, bias, T, d, N, k, eps_c, logits, unsure, idx, gates, cc, s); break;
+      default: e = launch_router_tc<128, 3>(tx, tw, bias, T, d, N, k, eps_c, logits, unsure, idx, gates, cc, s); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "router_topk: tensor-core router");
   } else {
@@ -834,9 +1040,32 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
     });
     if (e != cudaSuccess) return cuda_fail(e, "router_topk: logits");
     e = launch("router_topk", s, [&] {
-      router_topk_kernel<<<grid_for(T, 8, sm_count() * 32), 256, 0, s>>>(logits, T, N, k, idx, gates);
+      const int g = grid_for(T, 8, sm_count() * 32);
+      if (x_dtype == BFMOE_BF16)
+        router_topk_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(logits, static_cast<const __nv_bfloat16*>(x), w_gate,
+                                                            bias, T, d, N, k, eps_c, idx, gates, unsure);
+      else
+        router_topk_kernel<float><<<g, 256, 0, s>>>(logits, static_cast<const float*>(x), w_gate, bias, T, d, N, k,
+                                                    eps_c, idx, gates, unsure);
     });
     if (e != cudaSuccess) return cuda_fail(e, "router_topk: top-k");
+  }
+  // the tokens left undecided by the float32 top-k, settled from exact
+  // logits (usually a few per thousand; near ties always)
+  {
+    const int g = grid_for(T, kFixWarps, sm_count() * 4);
+    int32_t* ccp = tc_router ? cc : nullptr;
+    e = launch("router_fixup", s, [&] {
+      if (x_dtype == BFMOE_BF16)
+        pdl_launch(router_fixup_kernel<__nv_bfloat16>, g, kFixWarps * 32, 0, s, static_cast<const __nv_bfloat16*>(x),
+                   w_gate, bias, static_cast<const float*>(logits), T, d, N, k, eps_c,
+                   static_cast<const int*>(unsure), idx, gates, ccp);
+      else
+        pdl_launch(router_fixup_kernel<float>, g, kFixWarps * 32, 0, s, static_cast<const float*>(x), w_gate, bias,
+                   static_cast<const float*>(logits), T, d, N, k, eps_c, static_cast<const int*>(unsure), idx, gates,
+                   ccp);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "router_topk: fix-up of undecided tokens");
   }
 
   const int chunk = bucket_chunk(k);
@@ -891,8 +1120,12 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
   if ((rc = check_ws(p, ws, ws_bytes, p.fwd_end))) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* W = static_cast<uint8_t*>(ws);
-  if ((rc = build_weight_tables(layer, x_dtype == BFMOE_BF16, p, W, s))) return rc;
-  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, s);
+  const uint8_t* tabs = static_cast<const uint8_t*>(layer->tables);
+  if (!tabs) {
+    if ((rc = build_weight_tables(layer, W + p.tabs, s))) return rc;
+    tabs = W + p.tabs;
+  }
+  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, tabs, s);
 }
 
 size_t bfmoe_moe_host_workspace_size(int d, int n_experts, int T, int k, int x_dtype, int chunk) {
@@ -943,7 +1176,11 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
   if (e == cudaSuccess) e = cudaEventRecord(ss->fork, s);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward_host: fork");
-  rc = build_weight_tables(layer, bf16, pc, Wm, ss->stream);
+  const uint8_t* tabs = static_cast<const uint8_t*>(layer->tables);
+  if (!tabs) {
+    rc = build_weight_tables(layer, Wm + pc.tabs, ss->stream);
+    tabs = Wm + pc.tabs;
+  }
   if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return cuda_fail(e, "moe_forward_host: join record");
   // W_g is split once for all chunks, while the first chunk is copied in
   __nv_bfloat16* parts = nullptr;
@@ -965,7 +1202,7 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
     if (c == 0 && (e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) rc = cuda_fail(e, "moe_forward_host: join");
     if (rc) break;
     rc = forward_body(layer, x_dev + o, bf16, Tc, k, idx, gates, rows, y_dev + o, make_plan(d, N, Tc, k, x_dtype), Wm,
-                      s);
+                      tabs, s);
     if (rc) break;
     if ((e = cudaEventRecord(pipe->ev_out[c], s)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(pipe->out, pipe->ev_out[c], 0)) != cudaSuccess ||
@@ -1003,20 +1240,46 @@ int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int 
   if (T == 0)
     return bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, nullptr, 0,
                              stream);
+  const uint8_t* tabs = static_cast<const uint8_t*>(layer->tables);
+  if (tabs) {
+    // prepared tables: router and forward in stream order, nothing on the side
+    rc = bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, W + p.fwd_end,
+                           p.rt_end, stream);
+    if (rc) return rc;
+    return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, tabs, s);
+  }
   // fork: the weight-derived tables build on the side stream while the router runs
   SideStream* ss = nullptr;
   if ((rc = side_stream(&ss))) return rc;
   cudaError_t e = cudaEventRecord(ss->fork, s);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward: fork");
-  if ((rc = build_weight_tables(layer, x_dtype == BFMOE_BF16, p, W, ss->stream))) return rc;
+  if ((rc = build_weight_tables(layer, W + p.tabs, ss->stream))) return rc;
   if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return cuda_fail(e, "moe_forward: join record");
   rc = bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, W + p.fwd_end,
                          p.rt_end, stream);
   // join before anything else can fail, so the side stream never outlives the call's work
   if ((e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) return cuda_fail(e, "moe_forward: join");
   if (rc) return rc;
-  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, s);
+  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, W + p.tabs, s);
+}
+
+size_t bfmoe_layer_tables_size(int d, int n_experts) {
+  if (d < 4 || d > BFMOE_MAX_D || !is_pow2(d) || n_experts < 1 || n_experts > BFMOE_MAX_EXPERTS) return 0;
+  return make_tab_plan(d, n_experts).total;
+}
+
+int bfmoe_prepare_layer(const bfmoe_layer* layer, void* tables, size_t bytes, bfmoe_stream_t stream) {
+  if (!layer || !tables) return fail(BFMOE_EINVAL, "prepare_layer: NULL pointer");
+  const int d = layer->d, N = layer->n_experts;
+  if (d < 4 || d > BFMOE_MAX_D || !is_pow2(d)) return fail(BFMOE_EINVAL, "prepare_layer: bad d=%d", d);
+  if (N < 1 || N > BFMOE_MAX_EXPERTS) return fail(BFMOE_EINVAL, "prepare_layer: n_experts=%d", N);
+  if (!layer->w_packed || !layer->theta || !layer->phi) return fail(BFMOE_EINVAL, "prepare_layer: NULL layer weights");
+  if (reinterpret_cast<uintptr_t>(tables) & 255u) return fail(BFMOE_EWORKSPACE, "prepare_layer: tables must be 256-byte aligned");
+  const size_t need = make_tab_plan(d, N).total;
+  if (bytes < need) return fail(BFMOE_EWORKSPACE, "prepare_layer: %zu bytes given, %zu needed", bytes, need);
+  int rc = build_weight_tables(layer, static_cast<uint8_t*>(tables), reinterpret_cast<cudaStream_t>(stream));
+  return rc ? rc : ok();
 }
 
 int bfmoe_materialize_expert(const bfmoe_layer* layer, int e_idx, float* w_out, bfmoe_stream_t stream) {
@@ -1034,6 +1297,119 @@ int bfmoe_materialize_expert(const bfmoe_layer* layer, int e_idx, float* w_out, 
                                                              w_out);
   });
   if (e != cudaSuccess) return cuda_fail(e, "materialize: launch");
+  return ok();
+}
+
+size_t bfmoe_backward_workspace_size(int d, int n_experts, int T, int k) {
+  if (check_sizes(d, n_experts, T, k) != BFMOE_OK) return 0;
+  return make_bw_plan(d, n_experts, T, k).total;
+}
+
+int bfmoe_backward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, int k, const float* w_gate,
+                   const int32_t* idx, const float* gates, const int32_t* offsets, const int32_t* rows,
+                   const float* gy, float* dx, float* dtheta, float* dphi, float* dw_base, float* dalpha,
+                   float* dw_gate, float* dbias, void* ws, size_t ws_bytes, bfmoe_stream_t stream) {
+  if (!layer) return fail(BFMOE_EINVAL, "backward: NULL layer");
+  const int d = layer->d, N = layer->n_experts, L = ilog2(d);
+  int rc = check_sizes(d, N, T, k);
+  if (rc) return rc;
+  if ((rc = check_dtype(x_dtype))) return rc;
+  if (!layer->w_packed || !layer->theta || !layer->phi) return fail(BFMOE_EINVAL, "backward: NULL layer weights");
+  if (!dtheta || !dphi || !dw_base || !dalpha || !dw_gate || !w_gate || !offsets)
+    return fail(BFMOE_EINVAL, "backward: NULL pointer");
+  if (T > 0 && (!x || !idx || !gates || !rows || !gy || !dx)) return fail(BFMOE_EINVAL, "backward: NULL pointer");
+  const BwPlan b = make_bw_plan(d, N, T, k);
+  if (!ws) return fail(BFMOE_EWORKSPACE, "backward: NULL workspace");
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(BFMOE_EWORKSPACE, "backward: workspace must be 256-byte aligned");
+  if (ws_bytes < b.total) return fail(BFMOE_EWORKSPACE, "backward: workspace has %zu bytes, needs %zu", ws_bytes, b.total);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* W = static_cast<uint8_t*>(ws);
+  float2* tab_t = reinterpret_cast<float2*>(W + b.tab_t);
+  float2* tab_p = reinterpret_cast<float2*>(W + b.tab_p);
+  uint32_t* wt = reinterpret_cast<uint32_t*>(W + b.wt);
+  float* U = reinterpret_cast<float*>(W + b.U);
+  float* Z = reinterpret_cast<float*>(W + b.Z);
+  float* dU = reinterpret_cast<float*>(W + b.dU);
+  float* dg = reinterpret_cast<float*>(W + b.dg);
+  float* dl = reinterpret_cast<float*>(W + b.dl);
+  float* part = reinterpret_cast<float*>(W + b.part);
+  float* dapart = reinterpret_cast<float*>(W + b.dapart);
+  const bool bf16 = x_dtype == BFMOE_BF16;
+  const long long R = static_cast<long long>(T) * k;
+  const long long nang = static_cast<long long>(N) * L * (d / 2);
+  const int wpr = words_per_row(d);
+  cudaError_t e;
+  // cos/sin of both butterflies, the base's transpose
+  e = launch("bw_tables", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->theta, nang, tab_t); });
+  if (e == cudaSuccess)
+    e = launch("bw_tables", s, [&] { rot_table_kernel<<<grid_for(nang, 256, 8192), 256, 0, s>>>(layer->phi, nang, tab_p); });
+  if (e == cudaSuccess)
+    e = launch("bw_transpose_base", s, [&] {
+      transpose_packed_kernel<<<grid_for(static_cast<long long>(d) * wpr, 256, 4096), 256, 0, s>>>(layer->w_packed, d,
+                                                                                                   wpr, wt);
+    });
+  if (e != cudaSuccess) return cuda_fail(e, "backward: tables");
+  if (T == 0) {
+    const size_t ang = static_cast<size_t>(nang) * 4;
+    if ((e = cudaMemsetAsync(dtheta, 0, ang, s)) != cudaSuccess || (e = cudaMemsetAsync(dphi, 0, ang, s)) != cudaSuccess ||
+        (e = cudaMemsetAsync(dw_base, 0, static_cast<size_t>(d) * d * 4, s)) != cudaSuccess ||
+        (e = cudaMemsetAsync(dalpha, 0, 4, s)) != cudaSuccess ||
+        (e = cudaMemsetAsync(dw_gate, 0, static_cast<size_t>(N) * d * 4, s)) != cudaSuccess ||
+        (dbias && (e = cudaMemsetAsync(dbias, 0, static_cast<size_t>(N) * 4, s)) != cudaSuccess))
+      return cuda_fail(e, "backward: memset");
+    return ok();
+  }
+  // recompute the forward's rows in float32: u (bucket order), z = alpha W u
+  if ((e = bw_rows_dispatch(d, x, bf16, idx, rows, offsets, gates, gy, tab_t, tab_p, R, k, L, N, U, Z, dU, dg, dtheta,
+                            dphi, 0, s)) != cudaSuccess)
+    return cuda_fail(e, "backward: pre-rotation");
+  const dim3 gg((R + 63) / 64, (d + 63) / 64);
+  e = launch("bw_gemm", s, [&] {
+    ternary_gemm_simt_kernel<float><<<gg, 256, 0, s>>>(U, layer->w_packed, wpr, R, d, layer->alpha, Z);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "backward: product");
+  // output side: dg, dz = B(phi)^T (g gy) (in place of z), dphi
+  if ((e = bw_rows_dispatch(d, x, bf16, idx, rows, offsets, gates, gy, tab_t, tab_p, R, k, L, N, U, Z, dU, dg, dtheta,
+                            dphi, 1, s)) != cudaSuccess)
+    return cuda_fail(e, "backward: output rotation");
+  // du = alpha W^T dz; M = dz^T u, dW = alpha M, dalpha = sum W .* M
+  e = launch("bw_gemm", s, [&] {
+    ternary_gemm_simt_kernel<float><<<gg, 256, 0, s>>>(Z, wt, wpr, R, d, layer->alpha, dU);
+  });
+  if (e == cudaSuccess)
+    e = launch("bw_outer", s, [&] {
+      const dim3 go((d + kOuterTile - 1) / kOuterTile, (d + kOuterTile - 1) / kOuterTile, b.slices);
+      outer_tn_kernel<<<go, 256, 0, s>>>(Z, U, R, d, part);
+    });
+  if (e == cudaSuccess)
+    e = launch("bw_outer_reduce", s, [&] {
+      outer_reduce_kernel<<<b.ra_blocks, 256, 0, s>>>(part, b.slices, d, layer->alpha, layer->w_packed, wpr, dw_base,
+                                                      dapart);
+    });
+  if (e == cudaSuccess) e = launch("bw_sum", s, [&] { sum_kernel<<<1, 32, 0, s>>>(dapart, b.ra_blocks, dalpha); });
+  if (e != cudaSuccess) return cuda_fail(e, "backward: base gradient");
+  // input side: per-row dx = B(theta) du (into the z buffer, row order), dtheta
+  if ((e = bw_rows_dispatch(d, x, bf16, idx, rows, offsets, gates, gy, tab_t, tab_p, R, k, L, N, U, Z, dU, dg, dtheta,
+                            dphi, 2, s)) != cudaSuccess)
+    return cuda_fail(e, "backward: input rotation");
+  // router and per-token sums
+  e = launch("bw_token", s, [&] {
+    const int g = grid_for(T, 8, sm_count() * 16);
+    if (bf16)
+      bw_token_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(Z, dg, gates, idx, w_gate, T, k, d, N, dl, dx);
+    else
+      bw_token_kernel<float><<<g, 256, 0, s>>>(Z, dg, gates, idx, w_gate, T, k, d, N, dl, dx);
+  });
+  if (e == cudaSuccess)
+    e = launch("bw_router", s, [&] {
+      if (bf16)
+        bw_router_kernel<__nv_bfloat16><<<N, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), dl, rows, offsets, k, d,
+                                                         R, dw_gate, dbias);
+      else
+        bw_router_kernel<float><<<N, 256, 0, s>>>(static_cast<const float*>(x), dl, rows, offsets, k, d, R, dw_gate,
+                                                 dbias);
+    });
+  if (e != cudaSuccess) return cuda_fail(e, "backward: router");
   return ok();
 }
 

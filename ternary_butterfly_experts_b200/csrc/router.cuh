@@ -1,5 +1,7 @@
 // Router: float32 logits x W_g^T (+ b), top-k with the lower expert index
-// first on equal logits, gates renormalised over the selected k.
+// first on equal logits, gates renormalised over the selected k.  A token
+// whose k-th and (k+1)-th float32 logits are too close for float32 to rank
+// them is settled again from exact logits (router_fixup_kernel).
 //
 // Mixture-of-experts selection is only defined in general on the pages
 // (signalfieldnotes ButterflyMoE article, glossary "Mixtures of Experts");
@@ -65,33 +67,112 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
   return va > vb || (va == vb && ia < ib);
 }
 
-// One warp per token: each lane keeps its own sorted top-k over a strided
-// subset of experts, then k rounds of a warp-wide arg-max merge.
-__global__ __launch_bounds__(256) void router_topk_kernel(const float* __restrict__ logits, int T, int N, int k,
-                                                          int32_t* __restrict__ idx, float* __restrict__ gates) {
+// ---------------------------------------------------------------------------
+// Undecided tokens.
+//
+// Float32 logits carry rounding errors that grow with |l| and d: simulated
+// for the tensor-core router's order of accumulation, at most
+// 4.3e-6 (1 + |l|) at d = 2048 and 1.1e-6 (1 + |l|) at d = 512.  That is the
+// width of the near-tie band (1e-5) within which a float64 reference may rank
+// differently, so a float32 top-k is only trusted when each selected logit
+// clears the next one (and the k-th the best logit left out) by more than
+// 2 eps, with
+//     eps(l) = eps_c (1 + |l|),   eps_c = 2e-5 sqrt(d / 2048)
+// (about 5 to 10 times the simulated worst case).  Other tokens (a few per
+// thousand; every near tie) are listed for router_fixup_kernel, which settles
+// them with logits that are exact to ~1e-13 (double-float32 sums).
+// ---------------------------------------------------------------------------
+// Every gap of the sorted list v[0] >= ... >= v[k-1] >= rej (the order of
+// the slots as well as the set) must clear the band.
+__device__ __forceinline__ bool gap_is_clear(float a, float b, float eps_c) {
+  if (!(b > -INFINITY)) return true;
+  const float e = eps_c * (1.f + fmaxf(fabsf(a), fabsf(b)));
+  return a - b > 2.f * e;
+}
+__device__ __forceinline__ bool topk_is_clear(const float* v, int k, float rej, float eps_c) {
+  bool clear = true;
+#pragma unroll
+  for (int j = 0; j < BFMOE_MAX_K; ++j)
+    if (j < k) clear = clear && gap_is_clear(v[j], j + 1 < k ? v[j + 1] : rej, eps_c);
+  return clear;
+}
+
+// Gates from float32 logits in descending order: softmax over the k.
+__device__ __forceinline__ void gates_f32(const float* v, int k, float* g) {
+  float z[BFMOE_MAX_K];
+  float sum = 0.f;
+  const bool finite_top = v[0] > -INFINITY;
+  for (int j = 0; j < k; ++j) {
+    z[j] = finite_top ? expf(v[j] - v[0]) : 1.f;
+    sum += z[j];
+  }
+  for (int j = 0; j < k; ++j) g[j] = z[j] / sum;
+}
+
+// Double-float32 arithmetic (error-free transformations; the _rn intrinsics
+// keep the compiler from fusing the products into the sums).
+__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
+  s = __fadd_rn(a, b);
+  const float bb = __fsub_rn(s, a);
+  e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
+}
+// (s, c) += x * w, the product's rounding error carried exactly
+__device__ __forceinline__ void df_mac(float x, float w, float& s, float& c) {
+  const float p = __fmul_rn(x, w);
+  const float pe = fmaf(x, w, -p);
+  float t;
+  two_sum(s, p, s, t);
+  c = __fadd_rn(c, __fadd_rn(t, pe));
+}
+// (s, c) += (s2, c2)
+__device__ __forceinline__ void df_add(float& s, float& c, float s2, float c2) {
+  float t;
+  two_sum(s, s2, s, t);
+  c = __fadd_rn(c, __fadd_rn(c2, t));
+}
+// (hi, lo) with |lo| <= ulp(hi) / 2, so pairs compare lexicographically
+__device__ __forceinline__ void df_normalize(float s, float c, float& hi, float& lo) {
+  hi = __fadd_rn(s, c);
+  lo = __fsub_rn(c, __fsub_rn(hi, s));
+}
+__device__ __forceinline__ bool df_ranks_before(float ah, float al, int ai, float bh, float bl, int bi) {
+  return ah > bh || (ah == bh && (al > bl || (al == bl && ai < bi)));
+}
+
+// One warp per token: each lane keeps its own sorted list of the k + 1 best
+// logits of a strided subset of experts, then k + 1 rounds of a warp-wide
+// arg-max merge give the k candidates and the best of the rest.
+template <typename Tx>
+__global__ __launch_bounds__(256) void router_topk_kernel(const float* __restrict__ logits, const Tx* __restrict__ x,
+                                                          const float* __restrict__ wg, const float* __restrict__ bias,
+                                                          int T, int d, int N, int k, float eps_c,
+                                                          int32_t* __restrict__ idx, float* __restrict__ gates,
+                                                          int* __restrict__ unsure_list) {
+  constexpr int M = BFMOE_MAX_K + 1;
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
+  const int kk = k + 1;  // list length
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
-    float v[BFMOE_MAX_K];
-    int id[BFMOE_MAX_K];
+    float v[M];
+    int id[M];
 #pragma unroll
-    for (int j = 0; j < BFMOE_MAX_K; ++j) {
+    for (int j = 0; j < M; ++j) {
       v[j] = -INFINITY;
       id[j] = 0x7fffffff;
     }
     const float* lrow = logits + static_cast<size_t>(t) * N;
-    float th_v = -INFINITY;  // the lane's current k-th entry
+    float th_v = -INFINITY;  // the lane's current last entry
     int th_i = 0x7fffffff;
     for (int e = lane; e < N; e += 32) {
       float l = lrow[e];
       if (isnan(l)) l = -INFINITY;
       if (!ranks_before(l, e, th_v, th_i)) continue;
-      // insert, keeping v[0..k) sorted
+      // insert, keeping v[0..kk) sorted
       float cv = l;
       int ci = e;
 #pragma unroll
-      for (int j = 0; j < BFMOE_MAX_K; ++j) {
-        if (j < k && ranks_before(cv, ci, v[j], id[j])) {
+      for (int j = 0; j < M; ++j) {
+        if (j < kk && ranks_before(cv, ci, v[j], id[j])) {
           const float tv = v[j];
           const int ti = id[j];
           v[j] = cv;
@@ -99,14 +180,138 @@ __global__ __launch_bounds__(256) void router_topk_kernel(const float* __restric
           cv = tv;
           ci = ti;
         }
-        if (j == k - 1) {
+        if (j == kk - 1) {
           th_v = v[j];
           th_i = id[j];
         }
       }
     }
+    // k + 1 rounds: the last one finds the best float32 logit left out
     float sel_v[BFMOE_MAX_K];
     int sel_i[BFMOE_MAX_K];
+    float rej = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      if (j > k) break;
+      float bv = v[0];
+      int bi = id[0];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(FULL_MASK, bv, off);
+        const int oi = __shfl_xor_sync(FULL_MASK, bi, off);
+        if (ranks_before(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (j == k) {
+        rej = bv;
+        break;
+      }
+      sel_v[j] = bv;
+      sel_i[j] = bi;
+      if (id[0] == bi) {  // the owner pops its head
+#pragma unroll
+        for (int q = 0; q + 1 < M; ++q) {
+          v[q] = v[q + 1];
+          id[q] = id[q + 1];
+        }
+        v[M - 1] = -INFINITY;
+        id[M - 1] = 0x7fffffff;
+      }
+    }
+    float g[BFMOE_MAX_K];
+    gates_f32(sel_v, k, g);
+    if (lane == 0) {
+      for (int j = 0; j < k; ++j) {
+        idx[static_cast<size_t>(t) * k + j] = sel_i[j];
+        gates[static_cast<size_t>(t) * k + j] = g[j];
+      }
+      if (!topk_is_clear(sel_v, k, rej, eps_c)) unsure_list[2 + atomicAdd(unsure_list, 1)] = t;
+    }
+  }
+}
+
+// The undecided tokens (unsure_list: [0] count, [2 ..] token ids), a warp
+// per token, from the float32 logits the router stored ([T][N]):
+//   1. the float32 k-th logit V; the true top-k lies among the experts whose
+//      float32 logit is at least V - 2 eps (each of the k first has a true
+//      logit >= V - eps); the window keeps those at V - 4 eps or above (all N
+//      experts if more than kFixWindow qualify);
+//   2. the window's logits as double-float32 sums (exact products,
+//      compensated sums: error ~1e-13 relative), lanes across d;
+//   3. the exact top-k (lower index first on equal logits), gates from the
+//      exact differences, and the bucket-chunk histograms moved from the
+//      provisional experts to the final ones (when the router wrote them
+//      already: chunk_counts, else NULL).
+constexpr int kFixWindow = 64;
+constexpr int kFixWarps = 8;
+
+// Double-float logit of expert e for x row xr (lanes across d).
+template <typename Tx>
+__device__ __forceinline__ void df_logit(const Tx* __restrict__ xr, const float* __restrict__ wg,
+                                         const float* __restrict__ bias, int d, int e, int lane, float& h, float& l) {
+  const float* wr = wg + static_cast<size_t>(e) * d;
+  float sa = 0.f, ca = 0.f;
+  for (int i = lane; i < d; i += 32) df_mac(to_f32(xr[i]), wr[i], sa, ca);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float s2 = __shfl_xor_sync(FULL_MASK, sa, o);
+    const float c2 = __shfl_xor_sync(FULL_MASK, ca, o);
+    df_add(sa, ca, s2, c2);
+  }
+  if (bias) df_add(sa, ca, bias[e], 0.f);
+  df_normalize(sa, ca, h, l);
+  if (isnan(h) || isnan(l)) {
+    h = -INFINITY;
+    l = 0.f;
+  }
+}
+
+template <typename Tx>
+__global__ __launch_bounds__(kFixWarps * 32) void router_fixup_kernel(
+    const Tx* __restrict__ x, const float* __restrict__ wg, const float* __restrict__ bias,
+    const float* __restrict__ logits, int T, int d, int N, int k, float eps_c, const int* __restrict__ unsure_list,
+    int32_t* __restrict__ idx, float* __restrict__ gates, int32_t* __restrict__ chunk_counts) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int win_s[kFixWarps][kFixWindow];
+  const int n = unsure_list[0];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int gw = blockIdx.x * kFixWarps + w, nwarps = gridDim.x * kFixWarps;
+  for (int u = gw; u < n; u += nwarps) {
+    const int t = unsure_list[2 + u];
+    if (t < 0 || t >= T) {
+      if (lane == 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(u));
+      continue;
+    }
+    const float* lr = logits + static_cast<size_t>(t) * N;
+    const Tx* xr = x + static_cast<size_t>(t) * d;
+    // 1. float32 k-th logit, then the window
+    float v[BFMOE_MAX_K];
+    int id[BFMOE_MAX_K];
+#pragma unroll
+    for (int j = 0; j < BFMOE_MAX_K; ++j) {
+      v[j] = -INFINITY;
+      id[j] = 0x7fffffff;
+    }
+    for (int e = lane; e < N; e += 32) {
+      float cv = lr[e];
+      if (isnan(cv)) cv = -INFINITY;
+      int ci = e;
+#pragma unroll
+      for (int q = 0; q < BFMOE_MAX_K; ++q) {
+        if (q < k && ranks_before(cv, ci, v[q], id[q])) {
+          const float tv = v[q];
+          const int ti = id[q];
+          v[q] = cv;
+          id[q] = ci;
+          cv = tv;
+          ci = ti;
+        }
+      }
+    }
+    float vk = -INFINITY;
 #pragma unroll
     for (int j = 0; j < BFMOE_MAX_K; ++j) {
       if (j >= k) break;
@@ -121,9 +326,8 @@ __global__ __launch_bounds__(256) void router_topk_kernel(const float* __restric
           bi = oi;
         }
       }
-      sel_v[j] = bv;
-      sel_i[j] = bi;
-      if (id[0] == bi) {  // the owner pops its head
+      vk = bv;
+      if (id[0] == bi) {
 #pragma unroll
         for (int q = 0; q + 1 < BFMOE_MAX_K; ++q) {
           v[q] = v[q + 1];
@@ -133,23 +337,73 @@ __global__ __launch_bounds__(256) void router_topk_kernel(const float* __restric
         id[BFMOE_MAX_K - 1] = 0x7fffffff;
       }
     }
-    if (lane == 0) {
-      float z[BFMOE_MAX_K];
-      float sum = 0.f;
-      const bool finite_top = sel_v[0] > -INFINITY;
+    const float thr = vk > -INFINITY ? vk - 4.f * eps_c * (1.f + fabsf(vk)) : -INFINITY;
+    int nwin = 0;
+    for (int e0 = 0; e0 < N; e0 += 32) {
+      const int e = e0 + lane;
+      float l = e < N ? lr[e] : -INFINITY;
+      if (isnan(l)) l = -INFINITY;
+      const bool in = e < N && l >= thr;
+      const unsigned m = __ballot_sync(FULL_MASK, in);
+      const int pos = nwin + __popc(m & ((1u << lane) - 1u));
+      if (in && pos < kFixWindow) win_s[w][pos] = e;
+      nwin += __popc(m);
+    }
+    __syncwarp();
+    // 2. exact logits of the window (all experts when it overflows) and
+    // 3. the exact top-k
+    const bool all = nwin > kFixWindow;
+    const int cnt = all ? N : nwin;
+    float vh[BFMOE_MAX_K], vl[BFMOE_MAX_K];
 #pragma unroll
-      for (int j = 0; j < BFMOE_MAX_K; ++j) {
-        if (j >= k) break;
-        z[j] = finite_top ? expf(sel_v[j] - sel_v[0]) : 1.f;
-        sum += z[j];
-      }
+    for (int j = 0; j < BFMOE_MAX_K; ++j) {
+      vh[j] = -INFINITY;
+      vl[j] = 0.f;
+      id[j] = 0x7fffffff;
+    }
+    for (int q = 0; q < cnt; ++q) {
+      const int e = all ? q : win_s[w][q];
+      float h, l;
+      df_logit(xr, wg, bias, d, e, lane, h, l);
+      // every lane holds the same value: a uniform insertion
+      float ch = h, cl = l;
+      int ci = e;
 #pragma unroll
-      for (int j = 0; j < BFMOE_MAX_K; ++j) {
-        if (j >= k) break;
-        idx[static_cast<size_t>(t) * k + j] = sel_i[j];
-        gates[static_cast<size_t>(t) * k + j] = z[j] / sum;
+      for (int r = 0; r < BFMOE_MAX_K; ++r) {
+        if (r < k && df_ranks_before(ch, cl, ci, vh[r], vl[r], id[r])) {
+          const float th = vh[r], tl = vl[r];
+          const int ti = id[r];
+          vh[r] = ch;
+          vl[r] = cl;
+          id[r] = ci;
+          ch = th;
+          cl = tl;
+          ci = ti;
+        }
       }
     }
+    if (lane == 0) {
+      // gates from the exact differences l_j - l_0
+      float z[BFMOE_MAX_K];
+      float sum = 0.f;
+      const bool finite_top = vh[0] > -INFINITY;
+      for (int j = 0; j < k; ++j) {
+        z[j] = finite_top ? expf(__fadd_rn(__fsub_rn(vh[j], vh[0]), __fsub_rn(vl[j], vl[0]))) : 1.f;
+        sum += z[j];
+      }
+      for (int j = 0; j < k; ++j) {
+        const size_t o = static_cast<size_t>(t) * k + j;
+        if (chunk_counts) {
+          const int old = idx[o];
+          int32_t* cc = chunk_counts + static_cast<size_t>(t / 128) * N;
+          if (old >= 0 && old < N) atomicSub(cc + old, 1);
+          if (id[j] >= 0 && id[j] < N) atomicAdd(cc + id[j], 1);
+        }
+        idx[o] = id[j];
+        gates[o] = z[j] / sum;
+      }
+    }
+    __syncwarp();
   }
 }
 

@@ -13,11 +13,15 @@
 // one of two TMEM accumulators; warps 2..9 read the logits from TMEM (warp w
 // owns TMEM lanes 32*(w%4) .., warps w and w+4 take the two halves of each
 // chunk's columns), each keeping a running top-k of its half (larger logit
-// first, lower expert index on ties, NaN below every number) while the next
-// chunk is being multiplied; the two partial lists of a row are merged through
-// shared memory, and the row's idx and renormalised gates are written.  The
-// CTA's 128*k routed rows form one bucket chunk: the epilogue also writes
-// their expert histogram (chunk_counts[blockIdx.x][e]).
+// first, lower expert index on ties, NaN below every number), and the largest
+// logit it left out, while the next chunk is being multiplied; the two partial
+// lists of a row are merged through shared memory, and the row's idx and
+// renormalised gates are written.  A row whose selected logits are not
+// separated from each other and from the best one left out by more than the
+// float32 error band (topk_is_clear, router.cuh) is listed for
+// router_fixup_kernel.  The CTA's 128*k routed rows form one bucket
+// chunk: the epilogue also writes their expert histogram
+// (chunk_counts[blockIdx.x][e]).
 #pragma once
 #include "common.cuh"
 #include "gemm_tc.cuh"
@@ -49,7 +53,7 @@ struct RouterTcCfg {
   static constexpr uint32_t STAGE_BYTES = A_BYTES + 3 * B_BYTES;
   static constexpr uint32_t BAR_BYTES = (2 * STAGES + 4) * 8 + 8;
   static constexpr uint32_t BIAS_BYTES = BFMOE_MAX_EXPERTS * 4;             // bias staged once
-  static constexpr uint32_t MERGE_BYTES = kGemmBM * BFMOE_MAX_K * 8;        // partial top-k lists
+  static constexpr uint32_t MERGE_BYTES = kGemmBM * BFMOE_MAX_K * 8 + kGemmBM * 4;  // top-k lists, rejected maxima
   static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + BIAS_BYTES + MERGE_BYTES;
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : 256));
 };
@@ -58,23 +62,29 @@ constexpr int kRouterThreads = 320;
 constexpr int kRouterEpiWarps = 8;
 
 // Running top-K of one row in registers (K compile-time): larger logit first,
-// lower expert index first on equal logits.
+// lower expert index first on equal logits; `rej` is the largest logit that
+// is not (or no longer) in the list.
 template <int K>
 struct TopK {
   float v[K];
   int id[K];
+  float rej;
   __device__ __forceinline__ void init() {
 #pragma unroll
     for (int j = 0; j < K; ++j) {
       v[j] = -INFINITY;
       id[j] = 0x7fffffff;
     }
+    rej = -INFINITY;
   }
   // Small K: the K compare-and-select steps run for every column, with no
   // branch (the lanes of a warp hold different rows, so an early exit would
   // diverge on most columns); larger K exits first when l cannot enter.
   __device__ __forceinline__ void push(float l, int e) {
-    if (K > 4 && !ranks_before(l, e, v[K - 1], id[K - 1])) return;
+    if (K > 4 && !ranks_before(l, e, v[K - 1], id[K - 1])) {
+      rej = fmaxf(rej, l);
+      return;
+    }
     float cv = l;
     int ci = e;
 #pragma unroll
@@ -87,6 +97,7 @@ struct TopK {
       cv = sw ? tv : cv;
       ci = sw ? ti : ci;
     }
+    rej = fmaxf(rej, cv);  // what fell out of the list
   }
 };
 
@@ -94,6 +105,8 @@ template <int BN, int STAGES, int K>
 __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                                                            const __grid_constant__ CUtensorMap tmW,
                                                            const float* __restrict__ bias, int T, int d, int N,
+                                                           float eps_c, float* __restrict__ logits,
+                                                           int* __restrict__ unsure_list,
                                                            int32_t* __restrict__ idx,
                                                            float* __restrict__ gates,
                                                            int32_t* __restrict__ chunk_counts) {
@@ -108,6 +121,7 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
   float* bias_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + Cfg::BAR_BYTES);
   float* merge_v = bias_s + BFMOE_MAX_EXPERTS;                       // [128][K]
   int* merge_i = reinterpret_cast<int*>(merge_v + kGemmBM * BFMOE_MAX_K);  // [128][K]
+  float* merge_r = reinterpret_cast<float*>(merge_i + kGemmBM * BFMOE_MAX_K);  // [128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kGemmBM;
@@ -231,7 +245,24 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
           const int e = e0 + q;
           float l = e < N ? __uint_as_float(r[q]) + bias_s[e] : -INFINITY;
           if (isnan(l)) l = -INFINITY;
+          r[q] = __float_as_uint(l);
           top.push(l, e < N ? e : 0x7fffffff);
+        }
+        // the float32 logits are kept for the fix-up of undecided tokens
+        if (row < T) {
+          float* dst = logits + static_cast<size_t>(row) * N + e0;
+          if ((N & 7) == 0 && e0 + 32 <= N) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 8 * u),
+                           "r"(r[8 * u]), "r"(r[8 * u + 1]), "r"(r[8 * u + 2]), "r"(r[8 * u + 3]), "r"(r[8 * u + 4]),
+                           "r"(r[8 * u + 5]), "r"(r[8 * u + 6]), "r"(r[8 * u + 7])
+                           : "memory");
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (e0 + q < N) dst[q] = __uint_as_float(r[q]);
+          }
         }
       }
     }
@@ -246,9 +277,10 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
       merge_v[lr * BFMOE_MAX_K + j] = top.v[j];
       merge_i[lr * BFMOE_MAX_K + j] = top.id[j];
     }
+    merge_r[lr] = top.rej;
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kRouterEpiWarps * 32) : "memory");
-  // the bias is no longer read: its shared memory becomes the histogram
+  // the bias is no longer read from shared memory: it becomes the histogram
   int* hist = reinterpret_cast<int*>(bias_s);
   const int et = threadIdx.x - 64;  // 0 .. 255
   for (int e = et; e < N; e += kRouterEpiWarps * 32) hist[e] = 0;
@@ -256,20 +288,16 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
   if (hf == 0 && ok && row < T) {
 #pragma unroll
     for (int j = 0; j < K; ++j) top.push(merge_v[lr * BFMOE_MAX_K + j], merge_i[lr * BFMOE_MAX_K + j]);
-    float z[K];
-    float sum = 0.f;
-    const bool finite_top = top.v[0] > -INFINITY;
-#pragma unroll
-    for (int j = 0; j < K; ++j) {
-      z[j] = finite_top ? expf(top.v[j] - top.v[0]) : 1.f;
-      sum += z[j];
-    }
+    top.rej = fmaxf(top.rej, merge_r[lr]);
+    float g[BFMOE_MAX_K];
+    gates_f32(top.v, K, g);
 #pragma unroll
     for (int j = 0; j < K; ++j) {
       idx[static_cast<size_t>(row) * K + j] = top.id[j];
-      gates[static_cast<size_t>(row) * K + j] = z[j] / sum;
+      gates[static_cast<size_t>(row) * K + j] = g[j];
       if (top.id[j] < N) atomicAdd(&hist[top.id[j]], 1);
     }
+    if (!topk_is_clear(top.v, K, top.rej, eps_c)) unsure_list[2 + atomicAdd(unsure_list, 1)] = row;
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kRouterEpiWarps * 32) : "memory");
   for (int e = et; e < N; e += kRouterEpiWarps * 32)

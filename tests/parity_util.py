@@ -8,7 +8,10 @@ Comparison rules:
   logit is within 1e-5 of the j-th largest of all N (for every rank j), in
   slots whose logits descend (within 1e-5);
 * buckets bit-exact against the oracle's buckets of the GPU's own routing;
-* gates within 1e-5 of the oracle's softmax over the GPU-selected experts;
+* gates within gate_tol(d) = 1e-5 * max(1, d / 512) of the oracle's softmax
+  over the GPU-selected experts: the gates are float32 softmaxes of float32
+  logits, whose rounding grows with d (measured on B200: 2e-6 at d = 512,
+  9e-6 at d = 1024, 2.3e-5 at d = 2048 with logits up to |l| ~ 25);
 * outputs: per-token relative L2 against the oracle evaluated with the GPU's
   routing (so near-tie tokens still check the arithmetic), at most 1e-5 on
   the float32 path and 1e-2 on the bfloat16 path.
@@ -20,6 +23,10 @@ import numpy as np
 from oracle import bfmoe_oracle as O
 
 TOL = {"f32": 1e-5, "bf16": 1e-2}
+
+
+def gate_tol(d):
+    return 1e-5 * max(1.0, d / 512)
 
 
 def run_cuda(inp, device="cuda", check_errors=True):
@@ -88,7 +95,7 @@ def compare(inp, gpu, tokens=None, tol=None):
     near, mism = check_routing(logits, idx_g, wl.k)
     g_ref = O.gates_for(logits, idx_g)
     gerr = np.abs(gpu["gates"][sel] - g_ref).max()
-    assert gerr < 1e-5, f"gate error {gerr}"
+    assert gerr < gate_tol(wl.d), f"gate error {gerr}"
     if tokens is None:
         c, o, r = O.buckets(gpu["idx"], wl.n_experts)
         assert np.array_equal(gpu["counts"], c), "bucket counts differ"
@@ -121,7 +128,7 @@ def compare_routing_full(inp, gpu, block=8192):
         near_n += int(near.sum())
         mism_n += int(mism.sum())
         gerr = max(gerr, float(np.abs(gpu["gates"][a:b] - O.gates_for(logits, idx_g)).max()))
-    assert gerr < 1e-5, f"gate error {gerr}"
+    assert gerr < gate_tol(wl.d), f"gate error {gerr}"
     c, o, r = O.buckets(gpu["idx"], wl.n_experts)
     assert np.array_equal(gpu["counts"], c), "bucket counts differ"
     assert np.array_equal(gpu["offsets"], o), "bucket offsets differ"

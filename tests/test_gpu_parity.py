@@ -4,7 +4,7 @@ import pytest
 
 import workloads as W
 from oracle import bfmoe_oracle as O
-from tests.parity_util import compare, run_cuda
+from tests.parity_util import compare, compare_routing_full, run_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -103,27 +103,32 @@ def test_tiny_f32_workload_full():
 
 def test_pages_example_workload_full():
     inp = W.generate(W.WORKLOADS["d512_n64"])
-    compare(inp, run_cuda(inp))
+    stats = compare(inp, run_cuda(inp))
+    print(f"d512_n64: {stats}")
 
 
 def test_headline_workload_full():
     inp = W.generate(W.WORKLOADS["d512_n256"])
     stats = compare(inp, run_cuda(inp))
+    print(f"d512_n256: {stats}")
     assert stats["max_rel_l2"] < 1e-2
 
 
 @pytest.mark.parametrize("name", ["d1024_n256", "d2048_n1024"])
-def test_large_workloads_sampled(name):
+def test_large_workloads_full_routing_sampled_outputs(name):
+    """The two largest workloads at full size: every token's routing against
+    the oracle's float64 logits, the bucket arrays against the oracle's
+    buckets, and the outputs of a token sample through the oracle's
+    three-step experts (forming every expert densely would take too long)."""
     inp = W.generate(W.WORKLOADS[name])
     gpu = run_cuda(inp)
     T = inp.wl.tokens
-    sample = np.unique(np.concatenate([np.arange(4), np.random.default_rng(5).integers(0, T, 12), [T - 1]]))
-    compare(inp, gpu, tokens=sample)
-    # whole-output properties at full size: finite, buckets a permutation
+    near, mism, gerr = compare_routing_full(inp, gpu)
+    print(f"{name}: {near} near-tie tokens of {T} ({mism} routed differently), gate error {gerr:.2e}")
+    sample = np.unique(np.concatenate([np.arange(4), np.random.default_rng(5).integers(0, T, 44), [T - 1]]))
+    stats = compare(inp, gpu, tokens=sample)
+    print(f"{name}: sampled outputs max rel L2 {stats['max_rel_l2']:.3e}")
     assert np.isfinite(gpu["y"]).all()
-    rows = np.sort(gpu["rows"])
-    assert np.array_equal(rows, np.arange(T * inp.wl.k))
-    assert np.array_equal(np.diff(gpu["offsets"]), gpu["counts"])
 
 
 # -- the boundary's maximum sizes ------------------------------------------------------
@@ -273,3 +278,37 @@ def test_moe_forward_in_a_cuda_graph():
     m.bfmoe_check_device_error()
     assert np.array_equal(y.float().cpu().numpy().astype(np.float64), gpu["y"])
     del g
+
+
+# -- prepared weight tables ------------------------------------------------------
+
+@pytest.mark.parametrize("d,N,k,T,dt", [(512, 64, 2, 777, "bf16"), (1024, 16, 2, 200, "bf16"),
+                                        (64, 8, 2, 256, "f32"), (32, 4, 3, 50, "bf16")])
+def test_prepared_tables_give_identical_results(d, N, k, T, dt):
+    """bfmoe_prepare_layer once, then the calls read the tables: bit for bit
+    the per-call results, for the fused path, the separate kernels and the
+    small-d path."""
+    m = B()
+    wl = W.custom("pt", d=d, n_experts=N, k=k, tokens=T, dtype=dt, bias_var=0.5)
+    inp = W.generate(wl, seed=d + N)
+    gpu = run_cuda(inp)
+    layer = gpu["layer"]
+    x = gpu["x"]
+    wg = torch.from_numpy(inp.w_gate).cuda()
+    bias = torch.from_numpy(inp.bias).cuda()
+    code = m.BFMOE_BF16 if dt == "bf16" else m.BFMOE_F32
+    layer.prepare()
+    try:
+        ws = m.workspace(d, N, T, k, code)
+        idx = torch.from_numpy(gpu["idx"]).cuda()
+        gates = torch.from_numpy(gpu["gates"].astype(np.float32)).cuda()
+        offsets = torch.from_numpy(gpu["offsets"]).cuda()
+        rows = torch.from_numpy(gpu["rows"]).cuda()
+        y = m.bfmoe_forward(layer, x, k, idx, gates, offsets, rows, ws)
+        ws2 = torch.empty(m.bfmoe_moe_workspace_size(d, N, T, k, code), dtype=torch.uint8, device="cuda")
+        y2, _ = m.bfmoe_moe_forward(layer, x, wg, bias, k, ws2)
+        m.bfmoe_check_device_error()
+        for yy in (y, y2):
+            assert np.array_equal(yy.float().cpu().numpy().astype(np.float64), gpu["y"])
+    finally:
+        layer.unprepare()
