@@ -202,7 +202,7 @@ bool fused_path(int xdt, int d) { return xdt == BFMOE_BF16 && d >= 64 && d <= 51
 // ---------------------------------------------------------------------------
 struct Plan {
   // forward
-  size_t tabs, xrot, z, slot, fwd_end;
+  size_t tabs, xrot, z, slot, pad, fwd_end;
   // router
   size_t logits, chunk_counts, totals, wg_parts, unsure, rt_end;
   size_t total;
@@ -230,6 +230,7 @@ Plan make_plan(int d, int N, long long T, int k, int xdt) {
     p.z = take(static_cast<size_t>(R) * d * inter);
   }
   p.slot = take(static_cast<size_t>(R) * d * inter);
+  p.pad = take(static_cast<size_t>(N + 1) * 4);  // padded bucket offsets (fused path)
   p.fwd_end = off;
   off = 0;
   const long long nchunks = (R + bucket_chunk(k) - 1) / bucket_chunk(k);
@@ -542,8 +543,9 @@ int build_weight_tables(const bfmoe_layer* layer, uint8_t* tabs, cudaStream_t s)
 
 template <int D>
 cudaError_t launch_fused(const CUtensorMap& tb, const __nv_bfloat16* x, const int32_t* idx, const float* gates,
-                         const int32_t* rows, const float4* tq, const float4* pq, long long R, int k, int N,
-                         float alpha, __nv_bfloat16* slot, cudaStream_t s) {
+                         const int32_t* rows, const int32_t* offsets, int32_t* pad_off, const float4* tq,
+                         const float4* pq, long long R, int k, int N, float alpha, __nv_bfloat16* slot,
+                         cudaStream_t s) {
   using C = FusedCfg<D>;
   static std::atomic<uint64_t> done{0};
   if (needs_attr(done)) {
@@ -552,11 +554,16 @@ cudaError_t launch_fused(const CUtensorMap& tb, const __nv_bfloat16* x, const in
     if (e != cudaSuccess) return e;
     attr_set(done);
   }
-  const long long tiles = (R + kGemmBM - 1) / kGemmBM;
+  // the buckets padded to multiples of 32 rows (bucket_pad_kernel)
+  cudaError_t e = launch("bucket_pad", s, [&] {
+    pdl_launch(bucket_pad_kernel, 1, 1024, static_cast<size_t>(N + 1) * 4, s, offsets, N, pad_off);
+  });
+  if (e != cudaSuccess) return e;
+  const long long tiles = (R + 31LL * N + kGemmBM - 1) / kGemmBM;  // at most
   const int grid = static_cast<int>(std::min<long long>(tiles, sm_count()));
   return launch("fused_expert", s, [&] {
-    pdl_launch(fused_expert_kernel<D>, grid, kFusedThreads, C::SMEM_BYTES, s, tb, x, idx, gates, rows, tq, pq, R, k,
-               N, alpha, slot);
+    pdl_launch(fused_expert_kernel<D>, grid, kFusedThreads, C::SMEM_BYTES, s, tb, x, idx, gates, rows, offsets,
+               static_cast<const int32_t*>(pad_off), tq, pq, R, k, N, alpha, slot);
   });
 }
 
@@ -580,8 +587,8 @@ cudaError_t launch_combine(bool bf16, bool fast, const void* slot, int T, int k,
 // Pre-rotation, ternary product, post-rotation with gates, combine.  `tabs`
 // holds the weight tables (TabPlan), built per call or prepared once.
 int forward_body(const bfmoe_layer* layer, const void* x, bool bf16, int T, int k, const int32_t* idx,
-                 const float* gates, const int32_t* rows, void* y, const Plan& p, uint8_t* W, const uint8_t* tabs,
-                 cudaStream_t s) {
+                 const float* gates, const int32_t* offsets, const int32_t* rows, void* y, const Plan& p, uint8_t* W,
+                 const uint8_t* tabs, cudaStream_t s) {
   const int d = layer->d, N = layer->n_experts, L = ilog2(d);
   const TabPlan tp = make_tab_plan(d, N);
   const float2* tab_t = reinterpret_cast<const float2*>(tabs + tp.theta);
@@ -595,16 +602,17 @@ int forward_body(const bfmoe_layer* layer, const void* x, bool bf16, int T, int 
 
   if (fused_path(bf16 ? BFMOE_BF16 : BFMOE_F32, d)) {
     CUtensorMap tb;
-    if (!make_tmap_bf16(&tb, wbf, d, d, std::min(d, 256))) return fail(BFMOE_ECUDA, "forward: tensor map encoding failed");
+    if (!make_tmap_bf16(&tb, wbf, d, d, std::min(d, 128))) return fail(BFMOE_ECUDA, "forward: tensor map encoding failed");
     const auto* xb = static_cast<const __nv_bfloat16*>(x);
     const auto* tq = reinterpret_cast<const float4*>(tab_t);
     const auto* pq = reinterpret_cast<const float4*>(tabs + tp.phi_pq);
     auto* sb = static_cast<__nv_bfloat16*>(slot);
+    int32_t* pad = reinterpret_cast<int32_t*>(W + p.pad);
     switch (d) {
-      case 64: e = launch_fused<64>(tb, xb, idx, gates, rows, tq, pq, R, k, N, layer->alpha, sb, s); break;
-      case 128: e = launch_fused<128>(tb, xb, idx, gates, rows, tq, pq, R, k, N, layer->alpha, sb, s); break;
-      case 256: e = launch_fused<256>(tb, xb, idx, gates, rows, tq, pq, R, k, N, layer->alpha, sb, s); break;
-      default: e = launch_fused<512>(tb, xb, idx, gates, rows, tq, pq, R, k, N, layer->alpha, sb, s); break;
+      case 64: e = launch_fused<64>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, s); break;
+      case 128: e = launch_fused<128>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, s); break;
+      case 256: e = launch_fused<256>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, s); break;
+      default: e = launch_fused<512>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, s); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "forward: fused expert kernel");
     e = launch_combine(true, true, slot, T, k, d, y, s);
@@ -1125,7 +1133,7 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
     if ((rc = build_weight_tables(layer, W + p.tabs, s))) return rc;
     tabs = W + p.tabs;
   }
-  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, tabs, s);
+  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, tabs, s);
 }
 
 size_t bfmoe_moe_host_workspace_size(int d, int n_experts, int T, int k, int x_dtype, int chunk) {
@@ -1201,8 +1209,8 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
                           Wm + pc.fwd_end, pc.rt_end, s, parts);
     if (c == 0 && (e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) rc = cuda_fail(e, "moe_forward_host: join");
     if (rc) break;
-    rc = forward_body(layer, x_dev + o, bf16, Tc, k, idx, gates, rows, y_dev + o, make_plan(d, N, Tc, k, x_dtype), Wm,
-                      tabs, s);
+    rc = forward_body(layer, x_dev + o, bf16, Tc, k, idx, gates, offsets, rows, y_dev + o,
+                      make_plan(d, N, Tc, k, x_dtype), Wm, tabs, s);
     if (rc) break;
     if ((e = cudaEventRecord(pipe->ev_out[c], s)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(pipe->out, pipe->ev_out[c], 0)) != cudaSuccess ||
@@ -1246,7 +1254,7 @@ int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int 
     rc = bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, W + p.fwd_end,
                            p.rt_end, stream);
     if (rc) return rc;
-    return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, tabs, s);
+    return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, tabs, s);
   }
   // fork: the weight-derived tables build on the side stream while the router runs
   SideStream* ss = nullptr;
@@ -1261,7 +1269,7 @@ int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int 
   // join before anything else can fail, so the side stream never outlives the call's work
   if ((e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) return cuda_fail(e, "moe_forward: join");
   if (rc) return rc;
-  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, rows, y, p, W, W + p.tabs, s);
+  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, W + p.tabs, s);
 }
 
 size_t bfmoe_layer_tables_size(int d, int n_experts) {

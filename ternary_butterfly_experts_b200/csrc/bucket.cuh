@@ -73,17 +73,18 @@ __global__ __launch_bounds__(1024) void bucket_scan_kernel(int32_t* __restrict__
     }
 }
 
-// Exclusive prefix sum of totals[0..N) into off[0..N] (shared memory), by a
+// Exclusive prefix sum of val(0..N) into off[0..N] (shared memory), by a
 // block of any multiple of 32 threads up to 1024; thread i sums experts
 // i*per .. i*per + per - 1.
-__device__ __forceinline__ void block_exclusive_scan(const int32_t* __restrict__ totals, int N, int* off) {
+template <class F>
+__device__ __forceinline__ void block_exclusive_scan(F val, int N, int* off) {
   __shared__ int warp_sum[32];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
   const int per = (N + blockDim.x - 1) / blockDim.x;
   int local = 0;
   for (int q = 0; q < per; ++q) {
     const int e = tid * per + q;
-    local += e < N ? totals[e] : 0;
+    local += e < N ? val(e) : 0;
   }
   int incl = local;
 #pragma unroll
@@ -109,7 +110,7 @@ __device__ __forceinline__ void block_exclusive_scan(const int32_t* __restrict__
     const int e = tid * per + q;
     if (e < N) {
       off[e] = run;
-      run += totals[e];
+      run += val(e);
     }
   }
   if (tid == static_cast<int>(blockDim.x) - 1) off[N] = run;
@@ -132,7 +133,7 @@ __global__ __launch_bounds__(1024) void bucket_scatter_kernel(const int32_t* __r
   for (int q = tid; q < N * 8; q += blockDim.x) reinterpret_cast<uint32_t*>(wcnt)[q] = 0u;
   pdl_wait();
   pdl_trigger();
-  block_exclusive_scan(totals, N, off);
+  block_exclusive_scan([&](int e) { return totals[e]; }, N, off);
   if (blockIdx.x == 0) {
     for (int e = tid; e <= N; e += blockDim.x) {
       offsets_out[e] = off[e];
@@ -162,6 +163,19 @@ __global__ __launch_bounds__(1024) void bucket_scatter_kernel(const int32_t* __r
     const int pos = off[e] + chunk_prefix[static_cast<size_t>(blockIdx.x) * N + e] + before + rank;
     rows[pos] = static_cast<int32_t>(r);
   }
+}
+
+// Offsets of the buckets padded to whole multiples of 32 rows (one block):
+// pad_off[e] = sum over e' < e of ceil32(offsets[e'+1] - offsets[e']);
+// pad_off[N] is the padded row count.  The fused expert kernel walks this
+// padded order, so that no warp's 32 rows mix experts.
+__global__ __launch_bounds__(1024) void bucket_pad_kernel(const int32_t* __restrict__ offsets, int N,
+                                                          int32_t* __restrict__ pad_off) {
+  extern __shared__ int poff[];  // [N+1]
+  pdl_wait();
+  pdl_trigger();
+  block_exclusive_scan([&](int e) { return (offsets[e + 1] - offsets[e] + 31) & ~31; }, N, poff);
+  for (int e = threadIdx.x; e <= N; e += blockDim.x) pad_off[e] = poff[e];
 }
 
 }  // namespace bfmoe

@@ -11,10 +11,13 @@
 //                 B(theta_e)^T in registers (the two warp layouts of
 //                 rotate_fast.cuh), round to bf16 and write them straight into
 //                 the MMA's A operand: 128 x d bf16 in shared memory, K-major
-//                 with the 128-byte swizzle that TMA would produce;
-//   warp 0 (lane 0) streams the bf16 base with TMA, 256 x 64 tiles, through
-//                 a two-stage ring;
-//   warp 1 (lane 0) issues tcgen05.mma (M = 128, N = min(d, 256), K = 16)
+//                 with the 128-byte swizzle that TMA would produce.  The rows
+//                 are claimed in units of 8 from a shared counter, and the
+//                 epilogue warps join in whenever they have no epilogue work
+//                 (the first tile, and the next tile once theirs is done);
+//   warp 0 (lane 0) streams the bf16 base with TMA, 128 x 64 tiles, through
+//                 a ring of 2 (d = 512) or 4 stages;
+//   warp 1 (lane 0) issues tcgen05.mma (M = 128, N = min(d, 128), K = 16)
 //                 into one fp32 accumulator of d TMEM columns: the tile's full
 //                 output rows;
 //   warps 10..17  (epilogue, two per TMEM lane quadrant, one thread per row)
@@ -44,8 +47,8 @@ namespace bfmoe {
 
 constexpr int kFusedProdWarps = 8;
 constexpr int kFusedEpiWarps = 8;
-constexpr int kFusedThreads = (2 + kFusedProdWarps + kFusedEpiWarps) * 32;
-constexpr int kFusedBStages = 2;
+constexpr int kFusedSimtWarps = kFusedProdWarps + kFusedEpiWarps;  // all of them produce A
+constexpr int kFusedThreads = (2 + kFusedSimtWarps) * 32;
 
 template <int D>
 struct FusedCfg {
@@ -53,21 +56,34 @@ struct FusedCfg {
   static constexpr int E = D / 32;
   using Gm = Geo<E>;
   static constexpr int L = Gm::L;
-  static constexpr int BN = D < 256 ? D : 256;  // MMA N
+  static constexpr int BN = D < 128 ? D : 128;  // MMA N (a 128-row W_base tile per stage)
   static constexpr int NH = D / BN;             // MMAs per k-step (N halves)
   static constexpr int NK = D / kGemmBK;        // k-blocks
   static constexpr int NCH = D / 32;            // 32-column chunks of a row
   static constexpr int PG = E >= 16 ? 2 : 4;    // rows per producer group
-  static constexpr int ROWS_PER_PROD = kGemmBM / kFusedProdWarps;
   static constexpr uint32_t A_KB_BYTES = kGemmBM * kGemmBK * 2;
   static constexpr uint32_t A_BYTES = NK * A_KB_BYTES;
   static constexpr uint32_t B_BYTES = BN * kGemmBK * 2;
+  static constexpr int BSTAGES = D >= 512 ? 2 : 4;  // W_base ring
+  // the theta quads of one expert, staged per tile for the producers
+  static constexpr int TABQ = tab_quads(E);
+  static constexpr uint32_t TAB_BYTES = TABQ * 16;
   static constexpr uint32_t PROD_BUF = D * 4;  // one float32 row: the layout switch
-  static constexpr uint32_t BAR_BYTES = (2 * kFusedBStages + 3 + 4) * 8 + 8;
-  static constexpr uint32_t SMEM_BYTES =
-      1024 + A_BYTES + kFusedBStages * B_BYTES + kFusedProdWarps * PROD_BUF + BAR_BYTES;
+  // per epilogue warp, two buffers of cos/sin quads staged from global memory:
+  // a chunk's stages 0..4 (5 x 8 quads) or a slice pair's stages 5.. (<= 32)
+  static constexpr int EPI_QUADS = 40;
+  // (also the layout-switch buffer when an epilogue warp helps produce A)
+  static constexpr uint32_t EPI_BUF = 2 * EPI_QUADS * 16 > D * 4 ? 2 * EPI_QUADS * 16 : D * 4;
+  // production of a tile's A is claimed in units of UNIT rows
+  static constexpr int UNIT = 8;
+  static constexpr int NUNITS = kGemmBM / UNIT;
+  static constexpr uint32_t BAR_BYTES = (2 * BSTAGES + 4 + 4) * 8 + 8 + 32;
+  static constexpr uint32_t SMEM_BYTES = 1024 + A_BYTES + BSTAGES * B_BYTES + kFusedProdWarps * PROD_BUF +
+                                         kFusedEpiWarps * EPI_BUF + TAB_BYTES + BAR_BYTES;
+  static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
+  static_assert((L - 5) * (NCH / 2) <= EPI_QUADS, "slice-pair quads fit the staging buffer");
   static constexpr uint32_t TMEM_COLS = D;
-  static_assert(ROWS_PER_PROD % PG == 0, "producer groups");
+  static_assert(UNIT % PG == 0, "producer groups");
 };
 
 // Byte offset, inside the A tile, of the 16-byte unit that holds elements
@@ -119,17 +135,72 @@ __device__ __forceinline__ void zero_a_row(uint8_t* A, int m, int lane) {
 }
 
 // Rows of a group in layout 2 straight from global memory (lane l reads
-// element q*32 + l of each row: 64 contiguous bytes per warp load).
+// element q*32 + l of each row: 64 contiguous bytes per warp load); a
+// negative token gives a row of zeros.
 template <int E, int G>
 __device__ __forceinline__ void load_x_rows_l2(const __nv_bfloat16* __restrict__ x, const int (&tok)[G],
                                                float (&v)[G][E], int lane) {
   constexpr int D = 32 * E;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const __nv_bfloat16* src = x + static_cast<size_t>(tok[g]) * D + lane;
+    const bool valid = tok[g] >= 0;
+    const __nv_bfloat16* src = x + static_cast<size_t>(valid ? tok[g] : 0) * D + lane;
 #pragma unroll
-    for (int q = 0; q < E; ++q) v[g][q] = __bfloat162float(src[q * 32]);
+    for (int q = 0; q < E; ++q) v[g][q] = valid ? __bfloat162float(src[q * 32]) : 0.f;
   }
+}
+
+// The kernel walks the buckets padded to whole multiples of 32 rows
+// (bucket_pad_kernel): padded position P lies in expert e's segment
+// [pad_off[e], pad_off[e+1]); it holds bucket position offsets[e] + P -
+// pad_off[e] when that is below the bucket's end, else nothing.  So the 32
+// rows of a TMEM lane quadrant, and the 8 rows of a production unit, never
+// mix experts.  Returns expert -1 past the last segment, position -1 for
+// padding.  The row's routing is checked against the segment's expert.
+// Expert whose padded segment holds position P (-1 past the last one).
+__device__ __forceinline__ int pad_expert(long long P, const int32_t* __restrict__ pad_off, int N) {
+  if (P >= pad_off[N]) return -1;
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pad_off[mid] <= P) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Untiled bulk copy global -> shared (no multicast); completes on bar.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+struct PadRow {
+  int e, row;  // expert; routed row r = t*k + j (or -1)
+};
+__device__ __forceinline__ PadRow pad_row(long long P, const int32_t* __restrict__ pad_off,
+                                          const int32_t* __restrict__ offsets, const int32_t* __restrict__ rows,
+                                          const int32_t* __restrict__ idx, long long R, int N) {
+  PadRow pr{-1, -1};
+  if (P >= pad_off[N]) return pr;
+  int lo = 0, hi = N - 1;  // the last e with pad_off[e] <= P
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pad_off[mid] <= P) lo = mid;
+    else hi = mid - 1;
+  }
+  pr.e = lo;
+  const long long local = P - pad_off[lo];
+  const long long b0 = offsets[lo], b1 = offsets[lo + 1];
+  if (b0 + local < b1) {
+    const long long p = b0 + local;
+    const int r = p >= 0 && p < R ? rows[p] : -1;
+    if (r >= 0 && r < R && idx[r] == lo) pr.row = r;
+    else report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
+  }
+  return pr;
 }
 
 // B(theta)^T of G rows held in layout 2; leaves them in layout 1.
@@ -148,19 +219,21 @@ __device__ __forceinline__ void rot_fwd(float& a, float& b, float c, float s) {
   a = na;
 }
 
-// Stages 0..4 of B(phi) on one 32-column chunk j of a row (thread = row).
-// tp: the row's expert table, [L][D/4] pair quads.
-template <int D>
-__device__ __forceinline__ void epi_chunk_stages(float (&v)[32], const float4* __restrict__ tp, int j) {
+// Stages 0..4 of B(phi) on one 32-column chunk of a row (thread = row).
+// t[s * stride + u] holds the pair quad of the chunk's local rotations 2u and
+// 2u+1 in stage s: the row's expert table in global memory (stride d/4, t at
+// the chunk's first quad) or the warp's staged copy in shared memory
+// (stride 8).
+template <int D, bool SHARED>
+__device__ __forceinline__ void epi_chunk_stages(float (&v)[32], const float4* __restrict__ t, int stride) {
   constexpr int L = FusedCfg<D>::L;
   constexpr int S5 = L < 5 ? L : 5;
 #pragma unroll
   for (int s = 0; s < S5; ++s) {
     const int h = 1 << s;
-    const float4* t = tp + s * (D / 4) + 8 * j;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const float4 q = __ldg(t + u);
+      const float4 q = SHARED ? t[s * stride + u] : __ldg(t + s * stride + u);
       // local rotations 2u and 2u+1 of this chunk: lower elements i0, i1
       const int r0 = 2 * u, r1 = 2 * u + 1;
       const int i0 = ((r0 >> s) << (s + 1)) | (r0 & (h - 1));
@@ -184,39 +257,200 @@ __device__ __forceinline__ void epi_chunk_stages(float (&v)[32], const float4* _
   }
 }
 
+// Stages 5..L-1 of B(phi) on the column slices c and c+1 of a row:
+// w[jj] = (column 32 jj + c, column 32 jj + c + 1).  The pair quad of stage s
+// and slice rotation mr is t[(s - 5) * st_s + mr * st_m].
+template <int D, bool SHARED>
+__device__ __forceinline__ void epi_slice_stages(float2 (&w)[D / 32], const float4* __restrict__ t, int st_s,
+                                                 int st_m) {
+  constexpr int L = FusedCfg<D>::L;
+  constexpr int NCH = D / 32;
+#pragma unroll
+  for (int s = 5; s < L; ++s) {
+    const int hh = 1 << (s - 5);
+#pragma unroll
+    for (int mr = 0; mr < NCH / 2; ++mr) {
+      // mr-th pair (jj, jj + hh) of the slice with bit (s-5) of jj clear
+      const int jj = ((mr >> (s - 5)) << (s - 4)) | (mr & (hh - 1));
+      const float4 q = SHARED ? t[(s - 5) * st_s + mr * st_m] : __ldg(t + (s - 5) * st_s + mr * st_m);
+      const float2 c2 = make_float2(q.x, q.y), s2 = make_float2(q.z, q.w);
+      const float2 a = w[jj], b = w[jj + hh];
+      w[jj] = __ffma2_rn(c2, a, __fmul2_rn(make_float2(-q.z, -q.w), b));
+      w[jj + hh] = __ffma2_rn(c2, b, __fmul2_rn(s2, a));
+    }
+  }
+}
+
+// What the producers of a CTA share.
+struct ProdCtx {
+  uint8_t* A;
+  int* claim;           // [2] unit counters (tile parity), [2] finished warps
+  uint64_t* a_full;     // producers -> MMA
+  uint64_t* mma_done;   // MMA -> producers (A free)
+  uint64_t* tab_full;   // the staged theta table has landed
+  const float4* tab_s;  // staged theta quads of expert *tab_ex
+  int* tab_ex;
+  int* tab_n;  // stagings issued (tab_full phases)
+  const __nv_bfloat16* x;
+  const int32_t* idx;
+  const int32_t* rows;
+  const int32_t* offsets;
+  const int32_t* pad_off;
+  const float4* tq_theta;
+  long long R, n_tiles;
+  int k, N, grid;
+};
+
+// Stage the theta quads of the expert that leads tile t (or none) and signal
+// tab_full.
+template <int D>
+__device__ __forceinline__ void stage_theta(const ProdCtx& c, long long t) {
+  using C = FusedCfg<D>;
+  const int e = t < c.n_tiles ? pad_expert(t * kGemmBM, c.pad_off, c.N) : -1;
+  *c.tab_ex = e;
+  *c.tab_n += 1;
+  if (e >= 0) {
+    mbar_expect_tx(c.tab_full, C::TAB_BYTES);
+    bulk_load(const_cast<float4*>(c.tab_s), c.tq_theta + static_cast<size_t>(e) * C::TABQ, C::TAB_BYTES, c.tab_full);
+  } else {
+    mbar_arrive(c.tab_full);
+  }
+}
+
+// Produce tile t's A operand (the tile's i-th in this CTA): every CUDA-core
+// warp of the CTA calls this once per tile and claims units of UNIT rows from
+// a shared counter until none are left; a unit's rows are gathered, rotated
+// by B(theta_e)^T in groups of PG rows of one expert, rounded to bf16 and
+// stored in A.  The quads of the tile's leading expert come from shared
+// memory (staged by stage_theta), others from global memory.  With
+// wait_free, the stores, and in any case the arrival, first wait for the
+// previous tile's MMAs (A still holds their operand).  The last warp to
+// finish resets the counters for tile i + 2 and stages the next tile's
+// table, then every warp arrives on a_full.
+template <int D>
+__device__ __forceinline__ bool produce_tile(const ProdCtx& c, long long t, int i, bool wait_free, float* buf,
+                                             int lane) {
+  using C = FusedCfg<D>;
+  using Gm = typename C::Gm;
+  constexpr int E = C::E, PG = C::PG;
+  int* ctr = c.claim + (i & 1);
+  int* done = c.claim + 2 + (i & 1);
+  bool ok = true, free_ = !wait_free, have_tab = false;
+  int tab_e = -1;
+  while (ok) {
+    int u = 0;
+    if (lane == 0) u = atomicAdd(ctr, 1);
+    u = __shfl_sync(FULL_MASK, u, 0);
+    if (u >= C::NUNITS) break;
+    if (!have_tab) {
+      if (!mbar_wait(c.tab_full, i & 1u, 0x2800u)) {
+        ok = false;
+        break;
+      }
+      tab_e = *c.tab_ex;
+      have_tab = true;
+    }
+    const int r0 = u * C::UNIT;
+    const PadRow mine = lane < C::UNIT ? pad_row(t * kGemmBM + r0 + lane, c.pad_off, c.offsets, c.rows, c.idx, c.R,
+                                                 c.N)
+                                       : PadRow{-1, -1};
+    const int my_tok = mine.row >= 0 ? mine.row / c.k : -1;
+#pragma unroll 1
+    for (int g0 = 0; g0 < C::UNIT; g0 += PG) {
+      int tok[PG];
+#pragma unroll
+      for (int g = 0; g < PG; ++g) tok[g] = __shfl_sync(FULL_MASK, my_tok, g0 + g);
+      const int e0 = __shfl_sync(FULL_MASK, mine.e, g0);
+      const unsigned gm = ((1u << PG) - 1u) << g0;
+      const unsigned same = __ballot_sync(FULL_MASK, mine.e >= 0 && mine.e == e0) & gm;
+      float v[PG][E];
+      load_x_rows_l2<E, PG>(c.x, tok, v, lane);
+      if (same == gm) {
+        // one expert (padding rows are zeros and stay zeros)
+        const float4* tq = e0 == tab_e ? c.tab_s : c.tq_theta + static_cast<size_t>(e0) * C::TABQ;
+        pre_rotate_core<Gm, PG>(v, tq, buf, lane);
+      } else {
+        // rows past the last segment (zeros), or inconsistent routing: one at a time
+#pragma unroll
+        for (int g = 0; g < PG; ++g) {
+          const int e = __shfl_sync(FULL_MASK, mine.e, g0 + g);
+          float v1[1][E];
+#pragma unroll
+          for (int q = 0; q < E; ++q) v1[0][q] = v[g][q];
+          if (e >= 0) pre_rotate_core<Gm, 1>(v1, c.tq_theta + static_cast<size_t>(e) * C::TABQ, buf, lane);
+#pragma unroll
+          for (int q = 0; q < E; ++q) v[g][q] = e >= 0 ? v1[0][q] : 0.f;
+        }
+      }
+      if (!free_) {
+        if (!mbar_wait(c.mma_done, (i - 1) & 1u, 0x2500u)) {
+          ok = false;
+          break;
+        }
+        free_ = true;
+      }
+#pragma unroll
+      for (int g = 0; g < PG; ++g) store_a_row<D>(c.A, r0 + g0 + g, v[g], lane);
+    }
+  }
+  // a warp left without rows still waits for the previous tile's MMAs before
+  // it arrives: an arrival for tile i must not land in tile i-1's phase, and
+  // tile i+1's counters are only reset once every warp is past tile i-1
+  if (ok && !free_ && !mbar_wait(c.mma_done, (i - 1) & 1u, 0x2500u)) ok = false;
+  // every warp has seen this tile's table before the next one replaces it
+  if (ok && !have_tab && !mbar_wait(c.tab_full, i & 1u, 0x2800u)) ok = false;
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    if (atomicAdd(done, 1) == kFusedSimtWarps - 1) {
+      *ctr = 0;
+      *done = 0;
+      stage_theta<D>(c, t + c.grid);
+    }
+    mbar_arrive(c.a_full);
+  }
+  return ok;
+}
+
 template <int D>
 __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
     const __grid_constant__ CUtensorMap tmB, const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ idx,
-    const float* __restrict__ gates, const int32_t* __restrict__ rows, const float4* __restrict__ tq_theta,
-    const float4* __restrict__ pq_phi, long long R, int k, int N, float alpha, __nv_bfloat16* __restrict__ slot) {
+    const float* __restrict__ gates, const int32_t* __restrict__ rows, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ pad_off, const float4* __restrict__ tq_theta, const float4* __restrict__ pq_phi,
+    long long R, int k, int N, float alpha, __nv_bfloat16* __restrict__ slot) {
   using C = FusedCfg<D>;
-  using Gm = typename C::Gm;
-  constexpr int E = C::E;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_align1024(smem_raw);
   uint8_t* A = smem;
   uint8_t* Bs = smem + C::A_BYTES;
-  float* prod_buf = reinterpret_cast<float*>(Bs + kFusedBStages * C::B_BYTES);
-  uint64_t* bfull = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(prod_buf) + kFusedProdWarps * C::PROD_BUF);
-  uint64_t* bempty = bfull + kFusedBStages;
-  uint64_t* a_full = bempty + kFusedBStages;  // producers -> MMA (one arrival per producer warp)
+  float* prod_buf = reinterpret_cast<float*>(Bs + C::BSTAGES * C::B_BYTES);
+  float4* epi_buf = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(prod_buf) + kFusedProdWarps * C::PROD_BUF);
+  float4* tab_s = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(epi_buf) + kFusedEpiWarps * C::EPI_BUF);
+  uint64_t* bfull = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(tab_s) + C::TAB_BYTES);
+  uint64_t* bempty = bfull + C::BSTAGES;
+  uint64_t* a_full = bempty + C::BSTAGES;  // producers -> MMA (one arrival per producer warp)
   uint64_t* mma_done = a_full + 1;            // MMA -> producers (A free) and epilogue (accumulator ready)
   uint64_t* acc_empty = mma_done + 1;         // epilogue -> MMA (one arrival per epilogue warp)
   uint64_t* qbar = acc_empty + 1;             // [4]: the two epilogue warps of a lane quadrant
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 4);
+  uint64_t* tab_full = qbar + 4;              // staged theta table
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tab_full + 1);
+  int* claim = reinterpret_cast<int*>(tmem_slot + 2);  // [2] unit counters (tile parity), [2] finished warps
+  int* tab_ex = claim + 4;
+  int* tab_n = claim + 5;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long n_tiles = (R + kGemmBM - 1) / kGemmBM;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kFusedBStages; ++s) {
+    for (int s = 0; s < C::BSTAGES; ++s) {
       mbar_init(bfull + s, 1);
       mbar_init(bempty + s, 1);
     }
-    mbar_init(a_full, kFusedProdWarps);
+    mbar_init(a_full, kFusedSimtWarps);
+    for (int q = 0; q < 6; ++q) claim[q] = 0;
     mbar_init(mma_done, 1);
     mbar_init(acc_empty, kFusedEpiWarps);
     for (int q = 0; q < 4; ++q) mbar_init(qbar + q, 2);
+    mbar_init(tab_full, 1);
     mbar_fence_init();
     tma_prefetch_desc(&tmB);
   }
@@ -225,8 +459,12 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();  // routing and buckets come from the previous kernel
+  pdl_wait();  // routing and buckets come from the previous kernels
   pdl_trigger();
+  const long long n_tiles = (static_cast<long long>(pad_off[N]) + kGemmBM - 1) / kGemmBM;
+  const ProdCtx pc{A, claim, a_full, mma_done, tab_full, tab_s, tab_ex, tab_n, x, idx, rows, offsets, pad_off, tq_theta,
+                   R, n_tiles, k, N, static_cast<int>(gridDim.x)};
+  if (threadIdx.x == 0) stage_theta<D>(pc, blockIdx.x);
 
   if (warp == 0) {
     // ---- TMA: the bf16 base, k-block by k-block, for every tile -----------
@@ -236,9 +474,9 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
       for (long long t = blockIdx.x; t < n_tiles && alive; t += gridDim.x) {
         for (int h = 0; h < C::NH && alive; ++h) {
           for (int kb = 0; kb < C::NK; ++kb, ++it) {
-            const int s = it % kFusedBStages;
-            const uint32_t ph = (it / kFusedBStages) & 1u;
-            if (it >= kFusedBStages && !mbar_wait(bempty + s, ph ^ 1u, 0x2100u | s)) {
+            const int s = it % C::BSTAGES;
+            const uint32_t ph = (it / C::BSTAGES) & 1u;
+            if (it >= C::BSTAGES && !mbar_wait(bempty + s, ph ^ 1u, 0x2100u | s)) {
               alive = false;
               break;
             }
@@ -260,8 +498,8 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
         tc_fence_after();
         for (int h = 0; h < C::NH && alive; ++h) {
           for (int kb = 0; kb < C::NK; ++kb, ++it) {
-            const int s = it % kFusedBStages;
-            const uint32_t ph = (it / kFusedBStages) & 1u;
+            const int s = it % C::BSTAGES;
+            const uint32_t ph = (it / C::BSTAGES) & 1u;
             if (!mbar_wait(bfull + s, ph, 0x2400u | s)) {
               alive = false;
               break;
@@ -283,79 +521,76 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
     // ---- producers: gather, B(theta)^T, bf16 into A -------------------------
     const int pw = warp - 2;
     float* buf = prod_buf + pw * (C::PROD_BUF / 4);
-    constexpr int PG = C::PG;
     int i = 0;
-    for (long long t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
-      const long long pb = t * kGemmBM + pw * C::ROWS_PER_PROD;
-      const RowMeta mine = lane < C::ROWS_PER_PROD ? fetch_row_meta(rows, idx, nullptr, pb + lane, R, N)
-                                                   : RowMeta{-1, -1, 0.f};
-      const int my_tok = mine.row >= 0 ? mine.row / k : 0;
-      bool ok = true;
-#pragma unroll 1
-      for (int g0 = 0; g0 < C::ROWS_PER_PROD; g0 += PG) {
-        int tok[PG];
-#pragma unroll
-        for (int g = 0; g < PG; ++g) tok[g] = __shfl_sync(FULL_MASK, my_tok, g0 + g);
-        const int e0 = __shfl_sync(FULL_MASK, mine.ex, g0);
-        const unsigned gm = ((1u << PG) - 1u) << g0;
-        const unsigned same = __ballot_sync(FULL_MASK, mine.ex >= 0 && mine.ex == e0) & gm;
-        float v[PG][E];
-        load_x_rows_l2<E, PG>(x, tok, v, lane);
-        if (same == gm) {
-          pre_rotate_core<Gm, PG>(v, tq_theta + static_cast<size_t>(e0) * tab_quads(E), buf, lane);
-        } else {
-          // rows of different experts (or past the end): one at a time
-#pragma unroll
-          for (int g = 0; g < PG; ++g) {
-            const int e = __shfl_sync(FULL_MASK, mine.ex, g0 + g);
-            float v1[1][E];
-#pragma unroll
-            for (int q = 0; q < E; ++q) v1[0][q] = v[g][q];
-            if (e >= 0) pre_rotate_core<Gm, 1>(v1, tq_theta + static_cast<size_t>(e) * tab_quads(E), buf, lane);
-#pragma unroll
-            for (int q = 0; q < E; ++q) v[g][q] = e >= 0 ? v1[0][q] : 0.f;
-          }
-        }
-        // A is free once the previous tile's MMAs have completed
-        if (g0 == 0 && i >= 1 && !mbar_wait(mma_done, (i - 1) & 1u, 0x2500u)) {
-          ok = false;
-          break;
-        }
-#pragma unroll
-        for (int g = 0; g < PG; ++g) store_a_row<D>(A, pw * C::ROWS_PER_PROD + g0 + g, v[g], lane);
-      }
-      if (!ok) break;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(a_full);
-    }
+    for (long long t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i)
+      if (!produce_tile<D>(pc, t, i, i >= 1, buf, lane))
+        break;
   } else {
     // ---- epilogue: alpha, B(phi), gate; one thread per row ---------------
     const int qd = warp & 3;                                  // TMEM lane quadrant
-    const int wq = (warp - 2 - kFusedProdWarps) >> 2;         // which half of the work
+    const int ew = warp - 2 - kFusedProdWarps;                // epilogue warp 0..7
+    const int wq = ew >> 2;                                   // which half of the work
     const int m = qd * 32 + lane;                             // row within the tile
     const uint32_t trow = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    float4* ebuf = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(epi_buf) + ew * C::EPI_BUF);
+    constexpr int S5 = C::L < 5 ? C::L : 5;
+    constexpr int NB = (C::L - 5) * (C::NCH / 2);  // quads of a slice pair
+    float* pbuf = reinterpret_cast<float*>(ebuf);  // layout-switch buffer while producing
     int i = 0;
-    for (long long t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
-      const long long p = t * kGemmBM + m;
-      const RowMeta mt = p < R ? fetch_row_meta(rows, idx, gates, p, R, N) : RowMeta{-1, -1, 0.f};
+    if (blockIdx.x < n_tiles &&
+        !produce_tile<D>(pc, blockIdx.x, 0, false, pbuf, lane))
+      i = -1;
+    for (long long t = blockIdx.x; t < n_tiles && i >= 0; t += gridDim.x, ++i) {
+      const PadRow pr = pad_row(t * kGemmBM + m, pad_off, offsets, rows, idx, R, N);
+      const RowMeta mt{pr.row, pr.e, pr.row >= 0 ? gates[pr.row] : 0.f};
       const float4* tp = pq_phi + static_cast<size_t>(mt.ex >= 0 ? mt.ex : 0) * C::L * (D / 4);
+      // the quadrant's rows share one expert (padded buckets): its quads are
+      // staged into shared memory ahead of use, bypassing L1; else (past the
+      // last segment) each row reads its own
+      const int ex0 = __shfl_sync(FULL_MASK, mt.ex, 0);
+      const bool uni = __all_sync(FULL_MASK, mt.ex == ex0) && ex0 >= 0;
+      const float4* tpu = pq_phi + static_cast<size_t>(ex0 >= 0 ? ex0 : 0) * C::L * (D / 4);
+      auto stage_chunk = [&](int j, int b) {
+        for (int l = lane; l < S5 * 8; l += 32)
+          cp_async16(ebuf + b * C::EPI_QUADS + l, tpu + (l >> 3) * (D / 4) + 8 * j + (l & 7));
+        cp_async_commit();
+      };
+      auto stage_slice = [&](int c, int b) {
+        for (int l = lane; l < NB; l += 32)
+          cp_async16(ebuf + b * C::EPI_QUADS + l,
+                     tpu + (5 + l / (C::NCH / 2)) * (D / 4) + (c >> 1) + 16 * (l % (C::NCH / 2)));
+        cp_async_commit();
+      };
       if (!mbar_wait(mma_done, i & 1u, 0x2600u)) break;
       tc_fence_after();
       // stages 0..4 inside each 32-column chunk (the two warps take alternate chunks)
+      if (uni) stage_chunk(wq, 0);
+      int b = 0;
 #pragma unroll 1
-      for (int j = wq; j < C::NCH; j += 2) {
+      for (int j = wq; j < C::NCH; j += 2, b ^= 1) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(trow + 32 * j, r);
+        if (uni) {
+          if (j + 2 < C::NCH) {
+            stage_chunk(j + 2, b ^ 1);
+            cp_async_wait<1>();
+          } else {
+            cp_async_wait<0>();
+          }
+          __syncwarp();
+        }
         tmem_wait_ld();
         float v[32];
 #pragma unroll
         for (int q = 0; q < 32; ++q) v[q] = alpha * __uint_as_float(r[q]);
-        epi_chunk_stages<D>(v, tp, j);
+        if (uni) epi_chunk_stages<D, true>(v, ebuf + b * C::EPI_QUADS, 8);
+        else epi_chunk_stages<D, false>(v, tp + 8 * j, D / 4);
 #pragma unroll
         for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(v[q]);
         tmem_st_32x32b_x32(trow + 32 * j, r);
+        __syncwarp();  // buffer b is refilled two chunks later
       }
+      if (uni) stage_slice(16 * wq, 0);
       tmem_wait_st();
       // both warps of the quadrant have finished the chunk stages
       tc_fence_before();
@@ -365,8 +600,9 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
       tc_fence_after();
       // stages 5..L-1 on column slices c, c+32, ...; this warp takes the
       // slices c in [16 wq, 16 wq + 16), two at a time
+      b = 0;
 #pragma unroll 1
-      for (int c = 16 * wq; c < 16 * wq + 16; c += 2) {
+      for (int c = 16 * wq; c < 16 * wq + 16; c += 2, b ^= 1) {
         float2 w[C::NCH];
 #pragma unroll
         for (int jj = 0; jj < C::NCH; ++jj) {
@@ -374,25 +610,22 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
           tmem_ld_32x32b_x2(trow + 32 * jj + c, a0, a1);
           w[jj] = make_float2(__uint_as_float(a0), __uint_as_float(a1));
         }
-        tmem_wait_ld();
-#pragma unroll
-        for (int s = 5; s < C::L; ++s) {
-          const int hh = 1 << (s - 5);
-          const float4* ts = tp + s * (D / 4) + (c >> 1);
-#pragma unroll
-          for (int mr = 0; mr < C::NCH / 2; ++mr) {
-            // mr-th pair (jj, jj + hh) of the slice with bit (s-5) of jj clear
-            const int jj = ((mr >> (s - 5)) << (s - 4)) | (mr & (hh - 1));
-            const float4 q = __ldg(ts + 16 * mr);  // rotations 32 mr + c, 32 mr + c + 1
-            const float2 c2 = make_float2(q.x, q.y), s2 = make_float2(q.z, q.w);
-            const float2 a = w[jj], b = w[jj + hh];
-            w[jj] = __ffma2_rn(c2, a, __fmul2_rn(make_float2(-q.z, -q.w), b));
-            w[jj + hh] = __ffma2_rn(c2, b, __fmul2_rn(s2, a));
+        if (uni) {
+          if (c + 2 < 16 * wq + 16) {
+            stage_slice(c + 2, b ^ 1);
+            cp_async_wait<1>();
+          } else {
+            cp_async_wait<0>();
           }
+          __syncwarp();
         }
+        tmem_wait_ld();
+        if (uni) epi_slice_stages<D, true>(w, ebuf + b * C::EPI_QUADS, C::NCH / 2, 1);
+        else epi_slice_stages<D, false>(w, tp + 5 * (D / 4) + (c >> 1), D / 4, 16);
 #pragma unroll
         for (int jj = 0; jj < C::NCH; ++jj)
           tmem_st_32x32b_x2(trow + 32 * jj + c, __float_as_uint(w[jj].x), __float_as_uint(w[jj].y));
+        __syncwarp();  // buffer b is refilled two slice pairs later
       }
       tmem_wait_st();
       // gated rows out: columns [16 wq, 16 wq + 16) of each chunk (the ones
@@ -402,7 +635,7 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
         uint32_t r[16];
         tmem_ld_32x32b_x16(trow + 32 * j + 16 * wq, r);
         tmem_wait_ld();
-        if (mt.ex >= 0) {
+        if (mt.row >= 0) {  // (padding rows have an expert but no row)
           uint32_t pk[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -420,10 +653,17 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
+      // then help produce the next tile's A (free: its MMAs have completed)
+      const long long tn = t + gridDim.x;
+      if (tn < n_tiles &&
+          !produce_tile<D>(pc, tn, i + 1, false, pbuf, lane))
+        break;
     }
   }
   tc_fence_before();
   __syncthreads();
+  // only the last staging can still be in flight (after an error exit)
+  if (threadIdx.x == 0 && *tab_n > 0) mbar_wait(tab_full, (*tab_n - 1) & 1u, 0x2a00u);
   if (warp == 0) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
