@@ -288,6 +288,19 @@ def run_ours(args, wl):
     def step():
         model(x, y=y)
 
+    if args.ncu_run:
+        # the launches a profiler captures: W warm-up steps, then K steps,
+        # eager (no graph), nothing else
+        for _ in range(args.warmup + args.steps):
+            step()
+        torch.cuda.synchronize()
+        B.bfmoe_check_device_error()
+        if rank == 0:
+            print(json.dumps({"ncu_run": wl.name, "steps": args.steps, "warmup": args.warmup}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
     def timed(n, fn, flush_l2=True):
         evs = []
         for _ in range(n):
@@ -511,6 +524,8 @@ def main():
     ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu-run", action="store_true",
+                    help="run warm-up + steps eagerly and exit (the command profiled under ncu)")
     ap.add_argument("--cpu-fraction", type=float, default=1.0,
                     help="fraction of the experts whose rows the CPU baseline evaluates")
     args = ap.parse_args()

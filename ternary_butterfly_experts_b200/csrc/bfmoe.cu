@@ -200,6 +200,10 @@ bool fused_path(int xdt, int d) { return xdt == BFMOE_BF16 && d >= 64 && d <= 51
 // ---------------------------------------------------------------------------
 // Workspace: router and forward share one buffer (stream-ordered).
 // ---------------------------------------------------------------------------
+// Positions of the padded bucket order that the fused expert kernel may
+// read: every bucket rounded up to 32 rows, the whole rounded up to tiles.
+long long pad_cap(long long R, int N) { return (R + 31LL * N + kGemmBM - 1) / kGemmBM * kGemmBM; }
+
 struct Plan {
   // forward
   size_t tabs, xrot, z, slot, pad, fwd_end;
@@ -230,7 +234,9 @@ Plan make_plan(int d, int N, long long T, int k, int xdt) {
     p.z = take(static_cast<size_t>(R) * d * inter);
   }
   p.slot = take(static_cast<size_t>(R) * d * inter);
-  p.pad = take(static_cast<size_t>(N + 1) * 4);  // padded bucket offsets (fused path)
+  // padded bucket offsets, padded row map and quadrant experts (fused path)
+  p.pad = take(static_cast<size_t>(N + 1) * 4 + static_cast<size_t>(pad_cap(R, N)) * 4 +
+               static_cast<size_t>(pad_cap(R, N) / 32) * 4);
   p.fwd_end = off;
   off = 0;
   const long long nchunks = (R + bucket_chunk(k) - 1) / bucket_chunk(k);
@@ -543,7 +549,7 @@ int build_weight_tables(const bfmoe_layer* layer, uint8_t* tabs, cudaStream_t s)
 
 template <int D>
 cudaError_t launch_fused(const CUtensorMap& tb, const __nv_bfloat16* x, const int32_t* idx, const float* gates,
-                         const int32_t* rows, const int32_t* offsets, int32_t* pad_off, const float4* tq,
+                         const int32_t* rows, const int32_t* offsets, int32_t* pad, const float4* tq,
                          const float4* pq, long long R, int k, int N, float alpha, __nv_bfloat16* slot,
                          cudaStream_t s) {
   using C = FusedCfg<D>;
@@ -554,16 +560,22 @@ cudaError_t launch_fused(const CUtensorMap& tb, const __nv_bfloat16* x, const in
     if (e != cudaSuccess) return e;
     attr_set(done);
   }
-  // the buckets padded to multiples of 32 rows (bucket_pad_kernel)
+  // the buckets padded to multiples of 32 rows, as a row map (bucket_pad_kernel)
+  const long long cap = pad_cap(R, N);
+  int32_t* pad_off = pad;
+  int32_t* pmap = pad + (N + 1);
+  int32_t* qex = pmap + cap;
   cudaError_t e = launch("bucket_pad", s, [&] {
-    pdl_launch(bucket_pad_kernel, 1, 1024, static_cast<size_t>(N + 1) * 4, s, offsets, N, pad_off);
+    const int g = grid_for(cap, 256, sm_count() * 8);
+    pdl_launch(bucket_pad_kernel, g, 256, static_cast<size_t>(N + 1) * 8, s, offsets, rows, idx, R, N, cap, pad_off,
+               pmap, qex);
   });
   if (e != cudaSuccess) return e;
-  const long long tiles = (R + 31LL * N + kGemmBM - 1) / kGemmBM;  // at most
-  const int grid = static_cast<int>(std::min<long long>(tiles, sm_count()));
+  const int grid = static_cast<int>(std::min<long long>(cap / kGemmBM, sm_count()));
   return launch("fused_expert", s, [&] {
-    pdl_launch(fused_expert_kernel<D>, grid, kFusedThreads, C::SMEM_BYTES, s, tb, x, idx, gates, rows, offsets,
-               static_cast<const int32_t*>(pad_off), tq, pq, R, k, N, alpha, slot);
+    pdl_launch(fused_expert_kernel<D>, grid, kFusedThreads, C::SMEM_BYTES, s, tb, x, gates,
+               static_cast<const int32_t*>(pmap), static_cast<const int32_t*>(qex),
+               static_cast<const int32_t*>(pad_off + N), tq, pq, k, alpha, slot);
   });
 }
 
@@ -1061,7 +1073,7 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
   // the tokens left undecided by the float32 top-k, settled from exact
   // logits (usually a few per thousand; near ties always)
   {
-    const int g = grid_for(T, kFixWarps, sm_count() * 4);
+    const int g = grid_for(T, kFixWarps, sm_count());
     int32_t* ccp = tc_router ? cc : nullptr;
     e = launch("router_fixup", s, [&] {
       if (x_dtype == BFMOE_BF16)

@@ -165,17 +165,52 @@ __global__ __launch_bounds__(1024) void bucket_scatter_kernel(const int32_t* __r
   }
 }
 
-// Offsets of the buckets padded to whole multiples of 32 rows (one block):
-// pad_off[e] = sum over e' < e of ceil32(offsets[e'+1] - offsets[e']);
-// pad_off[N] is the padded row count.  The fused expert kernel walks this
-// padded order, so that no warp's 32 rows mix experts.
-__global__ __launch_bounds__(1024) void bucket_pad_kernel(const int32_t* __restrict__ offsets, int N,
-                                                          int32_t* __restrict__ pad_off) {
-  extern __shared__ int poff[];  // [N+1]
+// The buckets padded to whole multiples of 32 rows, as a map from padded
+// position to routed row.  pad_off[e] = sum over e' < e of
+// ceil32(offsets[e'+1] - offsets[e']); pad_off[N] is the padded row count.
+// Padded position P in expert e's segment [pad_off[e], pad_off[e+1]) holds
+// bucket position offsets[e] + P - pad_off[e] when that is below the
+// bucket's end: pmap[P] is then its routed row (checked against idx), else
+// -1; qex[P / 32] is the expert of the 32 rows from P (-1 past the last
+// segment).  Every block scans the padded sizes itself (N <= 4096); the map
+// covers [0, p_cap), p_cap a multiple of 32 at least pad_off[N].  The fused
+// expert kernel walks this order, so that no warp's 32 rows mix experts.
+__global__ __launch_bounds__(256) void bucket_pad_kernel(const int32_t* __restrict__ offsets,
+                                                         const int32_t* __restrict__ rows,
+                                                         const int32_t* __restrict__ idx, long long R, int N,
+                                                         long long p_cap, int32_t* __restrict__ pad_off,
+                                                         int32_t* __restrict__ pmap, int32_t* __restrict__ qex) {
+  extern __shared__ int poff[];  // [N+1] padded offsets, then [N+1] offsets
+  int* off = poff + (N + 1);
   pdl_wait();
   pdl_trigger();
-  block_exclusive_scan([&](int e) { return (offsets[e + 1] - offsets[e] + 31) & ~31; }, N, poff);
-  for (int e = threadIdx.x; e <= N; e += blockDim.x) pad_off[e] = poff[e];
+  for (int e = threadIdx.x; e <= N; e += blockDim.x) off[e] = offsets[e];
+  __syncthreads();
+  block_exclusive_scan([&](int e) { return (off[e + 1] - off[e] + 31) & ~31; }, N, poff);
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e <= N; e += blockDim.x) pad_off[e] = poff[e];
+  const long long total = poff[N];
+  for (long long P = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; P < p_cap;
+       P += static_cast<long long>(gridDim.x) * blockDim.x) {
+    int e = -1, row = -1;
+    if (P < total) {
+      int lo = 0, hi = N - 1;  // the last e with poff[e] <= P
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (poff[mid] <= P) lo = mid;
+        else hi = mid - 1;
+      }
+      e = lo;
+      const long long b = off[e] + (P - poff[e]);
+      if (b < off[e + 1]) {
+        const int r = b >= 0 && b < R ? rows[b] : -1;
+        if (r >= 0 && r < R && idx[r] == e) row = r;
+        else report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(b));
+      }
+    }
+    pmap[P] = row;
+    if ((P & 31) == 0) qex[P >> 5] = e;
+  }
 }
 
 }  // namespace bfmoe

@@ -67,7 +67,7 @@ struct FusedCfg {
   static constexpr int BSTAGES = D >= 512 ? 2 : 4;  // W_base ring
   // the theta quads of one expert, staged per tile for the producers
   static constexpr int TABQ = tab_quads(E);
-  static constexpr uint32_t TAB_BYTES = TABQ * 16;
+  static constexpr uint32_t TAB_FULL = TABQ * 16;
   static constexpr uint32_t PROD_BUF = D * 4;  // one float32 row: the layout switch
   // per epilogue warp, two buffers of cos/sin quads staged from global memory:
   // a chunk's stages 0..4 (5 x 8 quads) or a slice pair's stages 5.. (<= 32)
@@ -77,9 +77,13 @@ struct FusedCfg {
   // production of a tile's A is claimed in units of UNIT rows
   static constexpr int UNIT = 8;
   static constexpr int NUNITS = kGemmBM / UNIT;
-  static constexpr uint32_t BAR_BYTES = (2 * BSTAGES + 4 + 4) * 8 + 8 + 32;
-  static constexpr uint32_t SMEM_BYTES = 1024 + A_BYTES + BSTAGES * B_BYTES + kFusedProdWarps * PROD_BUF +
-                                         kFusedEpiWarps * EPI_BUF + TAB_BYTES + BAR_BYTES;
+  static constexpr uint32_t BAR_BYTES = (2 * BSTAGES + 4 + 4 + NH) * 8 + 8 + 32;
+  static constexpr uint32_t SMEM_NO_TAB =
+      1024 + A_BYTES + BSTAGES * B_BYTES + kFusedProdWarps * PROD_BUF + kFusedEpiWarps * EPI_BUF + BAR_BYTES;
+  // the staged theta table where it fits (not at d = 512)
+  static constexpr bool USE_TAB = SMEM_NO_TAB + TAB_FULL <= 232448;
+  static constexpr uint32_t TAB_BYTES = USE_TAB ? TAB_FULL : 0;
+  static constexpr uint32_t SMEM_BYTES = SMEM_NO_TAB + TAB_BYTES;
   static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
   static_assert((L - 5) * (NCH / 2) <= EPI_QUADS, "slice-pair quads fit the staging buffer");
   static constexpr uint32_t TMEM_COLS = D;
@@ -151,22 +155,15 @@ __device__ __forceinline__ void load_x_rows_l2(const __nv_bfloat16* __restrict__
 }
 
 // The kernel walks the buckets padded to whole multiples of 32 rows
-// (bucket_pad_kernel): padded position P lies in expert e's segment
-// [pad_off[e], pad_off[e+1]); it holds bucket position offsets[e] + P -
-// pad_off[e] when that is below the bucket's end, else nothing.  So the 32
-// rows of a TMEM lane quadrant, and the 8 rows of a production unit, never
-// mix experts.  Returns expert -1 past the last segment, position -1 for
-// padding.  The row's routing is checked against the segment's expert.
-// Expert whose padded segment holds position P (-1 past the last one).
-__device__ __forceinline__ int pad_expert(long long P, const int32_t* __restrict__ pad_off, int N) {
-  if (P >= pad_off[N]) return -1;
-  int lo = 0, hi = N - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (pad_off[mid] <= P) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
+// (bucket_pad_kernel): position P holds routed row pmap[P] (-1: padding) of
+// expert qex[P / 32] (-1 past the last segment).  So the 32 rows of a TMEM
+// lane quadrant, and the 8 rows of a production unit, never mix experts.
+struct PadRow {
+  int e, row;  // expert; routed row r = t*k + j (or -1)
+};
+__device__ __forceinline__ PadRow pad_row(long long P, const int32_t* __restrict__ pmap,
+                                          const int32_t* __restrict__ qex) {
+  return PadRow{qex[P >> 5], pmap[P]};
 }
 
 // Untiled bulk copy global -> shared (no multicast); completes on bar.
@@ -175,32 +172,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                    smem_u32(dst)),
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
-}
-
-struct PadRow {
-  int e, row;  // expert; routed row r = t*k + j (or -1)
-};
-__device__ __forceinline__ PadRow pad_row(long long P, const int32_t* __restrict__ pad_off,
-                                          const int32_t* __restrict__ offsets, const int32_t* __restrict__ rows,
-                                          const int32_t* __restrict__ idx, long long R, int N) {
-  PadRow pr{-1, -1};
-  if (P >= pad_off[N]) return pr;
-  int lo = 0, hi = N - 1;  // the last e with pad_off[e] <= P
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (pad_off[mid] <= P) lo = mid;
-    else hi = mid - 1;
-  }
-  pr.e = lo;
-  const long long local = P - pad_off[lo];
-  const long long b0 = offsets[lo], b1 = offsets[lo + 1];
-  if (b0 + local < b1) {
-    const long long p = b0 + local;
-    const int r = p >= 0 && p < R ? rows[p] : -1;
-    if (r >= 0 && r < R && idx[r] == lo) pr.row = r;
-    else report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
-  }
-  return pr;
 }
 
 // B(theta)^T of G rows held in layout 2; leaves them in layout 1.
@@ -292,13 +263,11 @@ struct ProdCtx {
   int* tab_ex;
   int* tab_n;  // stagings issued (tab_full phases)
   const __nv_bfloat16* x;
-  const int32_t* idx;
-  const int32_t* rows;
-  const int32_t* offsets;
-  const int32_t* pad_off;
+  const int32_t* pmap;
+  const int32_t* qex;
   const float4* tq_theta;
-  long long R, n_tiles;
-  int k, N, grid;
+  long long n_tiles;
+  int k, grid;
 };
 
 // Stage the theta quads of the expert that leads tile t (or none) and signal
@@ -306,7 +275,7 @@ struct ProdCtx {
 template <int D>
 __device__ __forceinline__ void stage_theta(const ProdCtx& c, long long t) {
   using C = FusedCfg<D>;
-  const int e = t < c.n_tiles ? pad_expert(t * kGemmBM, c.pad_off, c.N) : -1;
+  const int e = C::USE_TAB && t < c.n_tiles ? c.qex[t * (kGemmBM / 32)] : -1;
   *c.tab_ex = e;
   *c.tab_n += 1;
   if (e >= 0) {
@@ -351,9 +320,7 @@ __device__ __forceinline__ bool produce_tile(const ProdCtx& c, long long t, int 
       have_tab = true;
     }
     const int r0 = u * C::UNIT;
-    const PadRow mine = lane < C::UNIT ? pad_row(t * kGemmBM + r0 + lane, c.pad_off, c.offsets, c.rows, c.idx, c.R,
-                                                 c.N)
-                                       : PadRow{-1, -1};
+    const PadRow mine = lane < C::UNIT ? pad_row(t * kGemmBM + r0 + lane, c.pmap, c.qex) : PadRow{-1, -1};
     const int my_tok = mine.row >= 0 ? mine.row / c.k : -1;
 #pragma unroll 1
     for (int g0 = 0; g0 < C::UNIT; g0 += PG) {
@@ -414,10 +381,10 @@ __device__ __forceinline__ bool produce_tile(const ProdCtx& c, long long t, int 
 
 template <int D>
 __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
-    const __grid_constant__ CUtensorMap tmB, const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ idx,
-    const float* __restrict__ gates, const int32_t* __restrict__ rows, const int32_t* __restrict__ offsets,
-    const int32_t* __restrict__ pad_off, const float4* __restrict__ tq_theta, const float4* __restrict__ pq_phi,
-    long long R, int k, int N, float alpha, __nv_bfloat16* __restrict__ slot) {
+    const __grid_constant__ CUtensorMap tmB, const __nv_bfloat16* __restrict__ x, const float* __restrict__ gates,
+    const int32_t* __restrict__ pmap, const int32_t* __restrict__ qex, const int32_t* __restrict__ pad_total,
+    const float4* __restrict__ tq_theta, const float4* __restrict__ pq_phi, int k, float alpha,
+    __nv_bfloat16* __restrict__ slot) {
   using C = FusedCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_align1024(smem_raw);
@@ -429,11 +396,12 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
   uint64_t* bfull = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(tab_s) + C::TAB_BYTES);
   uint64_t* bempty = bfull + C::BSTAGES;
   uint64_t* a_full = bempty + C::BSTAGES;  // producers -> MMA (one arrival per producer warp)
-  uint64_t* mma_done = a_full + 1;            // MMA -> producers (A free) and epilogue (accumulator ready)
+  uint64_t* mma_done = a_full + 1;            // MMA -> producers (A free)
   uint64_t* acc_empty = mma_done + 1;         // epilogue -> MMA (one arrival per epilogue warp)
   uint64_t* qbar = acc_empty + 1;             // [4]: the two epilogue warps of a lane quadrant
   uint64_t* tab_full = qbar + 4;              // staged theta table
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tab_full + 1);
+  uint64_t* acc_blk = tab_full + 1;           // [NH]: MMA -> epilogue, one N block of the accumulator ready
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_blk + C::NH);
   int* claim = reinterpret_cast<int*>(tmem_slot + 2);  // [2] unit counters (tile parity), [2] finished warps
   int* tab_ex = claim + 4;
   int* tab_n = claim + 5;
@@ -451,6 +419,7 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
     mbar_init(acc_empty, kFusedEpiWarps);
     for (int q = 0; q < 4; ++q) mbar_init(qbar + q, 2);
     mbar_init(tab_full, 1);
+    for (int q = 0; q < C::NH; ++q) mbar_init(acc_blk + q, 1);
     mbar_fence_init();
     tma_prefetch_desc(&tmB);
   }
@@ -461,10 +430,14 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
   const uint32_t tmem = *tmem_slot;
   pdl_wait();  // routing and buckets come from the previous kernels
   pdl_trigger();
-  const long long n_tiles = (static_cast<long long>(pad_off[N]) + kGemmBM - 1) / kGemmBM;
-  const ProdCtx pc{A, claim, a_full, mma_done, tab_full, tab_s, tab_ex, tab_n, x, idx, rows, offsets, pad_off, tq_theta,
-                   R, n_tiles, k, N, static_cast<int>(gridDim.x)};
+  const long long n_tiles = (static_cast<long long>(*pad_total) + kGemmBM - 1) / kGemmBM;
+  const ProdCtx pc{A,    claim, a_full,    mma_done, tab_full, tab_s, tab_ex, tab_n, x, pmap, qex, tq_theta,
+                   n_tiles, k,     static_cast<int>(gridDim.x)};
   if (threadIdx.x == 0) stage_theta<D>(pc, blockIdx.x);
+  // every CTA walks the base's (N block, k block) tiles from its own starting
+  // point, so that the CTAs do not all read the same L2 lines at once
+  const int b_h0 = static_cast<int>(blockIdx.x % C::NH);
+  const int b_kb0 = static_cast<int>((blockIdx.x / C::NH) % C::NK);
 
   if (warp == 0) {
     // ---- TMA: the bf16 base, k-block by k-block, for every tile -----------
@@ -472,8 +445,10 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
       int it = 0;
       bool alive = true;
       for (long long t = blockIdx.x; t < n_tiles && alive; t += gridDim.x) {
-        for (int h = 0; h < C::NH && alive; ++h) {
-          for (int kb = 0; kb < C::NK; ++kb, ++it) {
+        for (int h0 = 0; h0 < C::NH && alive; ++h0) {
+          const int h = (h0 + b_h0) % C::NH;
+          for (int kb0 = 0; kb0 < C::NK; ++kb0, ++it) {
+            const int kb = (kb0 + b_kb0) % C::NK;
             const int s = it % C::BSTAGES;
             const uint32_t ph = (it / C::BSTAGES) & 1u;
             if (it >= C::BSTAGES && !mbar_wait(bempty + s, ph ^ 1u, 0x2100u | s)) {
@@ -496,8 +471,10 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
         if (!mbar_wait(a_full, i & 1u, 0x2200u)) break;
         if (i >= 1 && !mbar_wait(acc_empty, (i - 1) & 1u, 0x2300u)) break;
         tc_fence_after();
-        for (int h = 0; h < C::NH && alive; ++h) {
-          for (int kb = 0; kb < C::NK; ++kb, ++it) {
+        for (int h0 = 0; h0 < C::NH && alive; ++h0) {
+          const int h = (h0 + b_h0) % C::NH;
+          for (int kb0 = 0; kb0 < C::NK; ++kb0, ++it) {
+            const int kb = (kb0 + b_kb0) % C::NK;
             const int s = it % C::BSTAGES;
             const uint32_t ph = (it / C::BSTAGES) & 1u;
             if (!mbar_wait(bfull + s, ph, 0x2400u | s)) {
@@ -510,9 +487,11 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
 #pragma unroll
             for (int kk = 0; kk < kGemmBK / 16; ++kk)
               mma_bf16_ss(tmem + static_cast<uint32_t>(h * C::BN), ad + 2u * kk, bd + 2u * kk, idesc,
-                          (kb | kk) != 0 ? 1u : 0u);
+                          (kb0 | kk) != 0 ? 1u : 0u);
             mma_commit(bempty + s);
           }
+          // the epilogue may start on this N block's columns
+          if (alive) mma_commit(acc_blk + h0);
         }
         if (alive) mma_commit(mma_done);
       }
@@ -541,7 +520,7 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
         !produce_tile<D>(pc, blockIdx.x, 0, false, pbuf, lane))
       i = -1;
     for (long long t = blockIdx.x; t < n_tiles && i >= 0; t += gridDim.x, ++i) {
-      const PadRow pr = pad_row(t * kGemmBM + m, pad_off, offsets, rows, idx, R, N);
+      const PadRow pr = pad_row(t * kGemmBM + m, pmap, qex);
       const RowMeta mt{pr.row, pr.e, pr.row >= 0 ? gates[pr.row] : 0.f};
       const float4* tp = pq_phi + static_cast<size_t>(mt.ex >= 0 ? mt.ex : 0) * C::L * (D / 4);
       // the quadrant's rows share one expert (padded buckets): its quads are
@@ -561,18 +540,31 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
                      tpu + (5 + l / (C::NCH / 2)) * (D / 4) + (c >> 1) + 16 * (l % (C::NCH / 2)));
         cp_async_commit();
       };
-      if (!mbar_wait(mma_done, i & 1u, 0x2600u)) break;
-      tc_fence_after();
-      // stages 0..4 inside each 32-column chunk (the two warps take alternate chunks)
-      if (uni) stage_chunk(wq, 0);
+      // stages 0..4 inside each 32-column chunk, N block by N block in the
+      // order the MMAs finish them (the two warps take alternate chunks)
+      constexpr int CPW = C::BN / 64 > 0 ? C::BN / 64 : 1;  // chunks of an N block per warp
+      auto chunk_of = [&](int n) {
+        const int h = (n / CPW + b_h0) % C::NH;
+        return h * (C::BN / 32) + 2 * (n % CPW) + wq;
+      };
+      if (uni) stage_chunk(chunk_of(0), 0);
       int b = 0;
+      bool alive = true;
 #pragma unroll 1
-      for (int j = wq; j < C::NCH; j += 2, b ^= 1) {
+      for (int n = 0; n < C::NCH / 2; ++n, b ^= 1) {
+        const int j = chunk_of(n);
+        if (n % CPW == 0) {
+          if (!mbar_wait(acc_blk + n / CPW, i & 1u, 0x2600u | (n / CPW))) {
+            alive = false;
+            break;
+          }
+          tc_fence_after();
+        }
         uint32_t r[32];
         tmem_ld_32x32b_x32(trow + 32 * j, r);
         if (uni) {
-          if (j + 2 < C::NCH) {
-            stage_chunk(j + 2, b ^ 1);
+          if (n + 1 < C::NCH / 2) {
+            stage_chunk(chunk_of(n + 1), b ^ 1);
             cp_async_wait<1>();
           } else {
             cp_async_wait<0>();
@@ -589,6 +581,10 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
         for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(v[q]);
         tmem_st_32x32b_x32(trow + 32 * j, r);
         __syncwarp();  // buffer b is refilled two chunks later
+      }
+      if (!alive) {
+        cp_async_wait<0>();
+        break;
       }
       if (uni) stage_slice(16 * wq, 0);
       tmem_wait_st();

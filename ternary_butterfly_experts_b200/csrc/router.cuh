@@ -139,6 +139,82 @@ __device__ __forceinline__ bool df_ranks_before(float ah, float al, int ai, floa
   return ah > bh || (ah == bh && (al > bl || (al == bl && ai < bi)));
 }
 
+// Four consecutive elements of a row as float32 (16-byte aligned for
+// float32, 8-byte for bfloat16).
+__device__ __forceinline__ void load4_f32(const float* p, float (&v)[4]) {
+  const float4 q = *reinterpret_cast<const float4*>(p);
+  v[0] = q.x;
+  v[1] = q.y;
+  v[2] = q.z;
+  v[3] = q.w;
+}
+__device__ __forceinline__ void load4_f32(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 q = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&q.x);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&q.y);
+  v[0] = __low2float(a);
+  v[1] = __high2float(a);
+  v[2] = __low2float(b);
+  v[3] = __high2float(b);
+}
+
+// Double-float logits of four experts at once (e[j] < 0: none; its result is
+// not used), so that the loads and sums of the four overlap.
+template <typename Tx>
+__device__ __forceinline__ void df_logits4(const Tx* __restrict__ xr, const float* __restrict__ wg,
+                                           const float* __restrict__ bias, int d, const int (&e)[4], int lane,
+                                           float (&h)[4], float (&l)[4]) {
+  const float* wr[4];
+  float sa[4], ca[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    wr[j] = wg + static_cast<size_t>(e[j] >= 0 ? e[j] : 0) * d;
+    sa[j] = 0.f;
+    ca[j] = 0.f;
+  }
+  const bool aligned = ((reinterpret_cast<uintptr_t>(xr) & (4 * sizeof(Tx) - 1)) |
+                        (reinterpret_cast<uintptr_t>(wg) & 15)) == 0;
+  if ((d & 127) == 0 && aligned) {
+    // four consecutive elements per lane and step: 16-byte weight loads
+    for (int i0 = 4 * lane; i0 < d; i0 += 128) {
+      float xv[4];
+      load4_f32(xr + i0, xv);
+      float4 w4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) w4[j] = *reinterpret_cast<const float4*>(wr[j] + i0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        df_mac(xv[0], w4[j].x, sa[j], ca[j]);
+        df_mac(xv[1], w4[j].y, sa[j], ca[j]);
+        df_mac(xv[2], w4[j].z, sa[j], ca[j]);
+        df_mac(xv[3], w4[j].w, sa[j], ca[j]);
+      }
+    }
+  } else {
+#pragma unroll 4
+    for (int i = lane; i < d; i += 32) {
+      const float xv = to_f32(xr[i]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) df_mac(xv, wr[j][i], sa[j], ca[j]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float s2 = __shfl_xor_sync(FULL_MASK, sa[j], o);
+      const float c2 = __shfl_xor_sync(FULL_MASK, ca[j], o);
+      df_add(sa[j], ca[j], s2, c2);
+    }
+    if (bias && e[j] >= 0) df_add(sa[j], ca[j], bias[e[j]], 0.f);
+    df_normalize(sa[j], ca[j], h[j], l[j]);
+    if (isnan(h[j]) || isnan(l[j])) {
+      h[j] = -INFINITY;
+      l[j] = 0.f;
+    }
+  }
+}
+
 // One warp per token: each lane keeps its own sorted list of the k + 1 best
 // logits of a strided subset of experts, then k + 1 rounds of a warp-wide
 // arg-max merge give the k candidates and the best of the rest.
@@ -233,7 +309,8 @@ __global__ __launch_bounds__(256) void router_topk_kernel(const float* __restric
 }
 
 // The undecided tokens (unsure_list: [0] count, [2 ..] token ids), a warp
-// per token, from the float32 logits the router stored ([T][N]):
+// per token, from the float32 logits the router stored ([T][N]) and its
+// provisional float32 top-k (idx):
 //   1. the float32 k-th logit V; the true top-k lies among the experts whose
 //      float32 logit is at least V - 2 eps (each of the k first has a true
 //      logit >= V - eps); the window keeps those at V - 4 eps or above (all N
@@ -246,27 +323,6 @@ __global__ __launch_bounds__(256) void router_topk_kernel(const float* __restric
 //      already: chunk_counts, else NULL).
 constexpr int kFixWindow = 64;
 constexpr int kFixWarps = 8;
-
-// Double-float logit of expert e for x row xr (lanes across d).
-template <typename Tx>
-__device__ __forceinline__ void df_logit(const Tx* __restrict__ xr, const float* __restrict__ wg,
-                                         const float* __restrict__ bias, int d, int e, int lane, float& h, float& l) {
-  const float* wr = wg + static_cast<size_t>(e) * d;
-  float sa = 0.f, ca = 0.f;
-  for (int i = lane; i < d; i += 32) df_mac(to_f32(xr[i]), wr[i], sa, ca);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float s2 = __shfl_xor_sync(FULL_MASK, sa, o);
-    const float c2 = __shfl_xor_sync(FULL_MASK, ca, o);
-    df_add(sa, ca, s2, c2);
-  }
-  if (bias) df_add(sa, ca, bias[e], 0.f);
-  df_normalize(sa, ca, h, l);
-  if (isnan(h) || isnan(l)) {
-    h = -INFINITY;
-    l = 0.f;
-  }
-}
 
 template <typename Tx>
 __global__ __launch_bounds__(kFixWarps * 32) void router_fixup_kernel(
@@ -287,58 +343,14 @@ __global__ __launch_bounds__(kFixWarps * 32) void router_fixup_kernel(
     }
     const float* lr = logits + static_cast<size_t>(t) * N;
     const Tx* xr = x + static_cast<size_t>(t) * d;
-    // 1. float32 k-th logit, then the window
-    float v[BFMOE_MAX_K];
-    int id[BFMOE_MAX_K];
-#pragma unroll
-    for (int j = 0; j < BFMOE_MAX_K; ++j) {
-      v[j] = -INFINITY;
-      id[j] = 0x7fffffff;
-    }
-    for (int e = lane; e < N; e += 32) {
-      float cv = lr[e];
-      if (isnan(cv)) cv = -INFINITY;
-      int ci = e;
-#pragma unroll
-      for (int q = 0; q < BFMOE_MAX_K; ++q) {
-        if (q < k && ranks_before(cv, ci, v[q], id[q])) {
-          const float tv = v[q];
-          const int ti = id[q];
-          v[q] = cv;
-          id[q] = ci;
-          cv = tv;
-          ci = ti;
-        }
-      }
-    }
-    float vk = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < BFMOE_MAX_K; ++j) {
-      if (j >= k) break;
-      float bv = v[0];
-      int bi = id[0];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(FULL_MASK, bv, off);
-        const int oi = __shfl_xor_sync(FULL_MASK, bi, off);
-        if (ranks_before(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      vk = bv;
-      if (id[0] == bi) {
-#pragma unroll
-        for (int q = 0; q + 1 < BFMOE_MAX_K; ++q) {
-          v[q] = v[q + 1];
-          id[q] = id[q + 1];
-        }
-        v[BFMOE_MAX_K - 1] = -INFINITY;
-        id[BFMOE_MAX_K - 1] = 0x7fffffff;
-      }
-    }
+    // 1. the float32 k-th logit V: the router's provisional k-th pick is
+    // the float32 top-k's last entry; then the window
+    const int ik = idx[static_cast<size_t>(t) * k + (k - 1)];
+    float vk = ik >= 0 && ik < N ? lr[ik] : -INFINITY;
+    if (isnan(vk)) vk = -INFINITY;
     const float thr = vk > -INFINITY ? vk - 4.f * eps_c * (1.f + fabsf(vk)) : -INFINITY;
     int nwin = 0;
+#pragma unroll 4
     for (int e0 = 0; e0 < N; e0 += 32) {
       const int e = e0 + lane;
       float l = e < N ? lr[e] : -INFINITY;
@@ -355,30 +367,37 @@ __global__ __launch_bounds__(kFixWarps * 32) void router_fixup_kernel(
     const bool all = nwin > kFixWindow;
     const int cnt = all ? N : nwin;
     float vh[BFMOE_MAX_K], vl[BFMOE_MAX_K];
+    int id[BFMOE_MAX_K];
 #pragma unroll
     for (int j = 0; j < BFMOE_MAX_K; ++j) {
       vh[j] = -INFINITY;
       vl[j] = 0.f;
       id[j] = 0x7fffffff;
     }
-    for (int q = 0; q < cnt; ++q) {
-      const int e = all ? q : win_s[w][q];
-      float h, l;
-      df_logit(xr, wg, bias, d, e, lane, h, l);
-      // every lane holds the same value: a uniform insertion
-      float ch = h, cl = l;
-      int ci = e;
+    for (int q0 = 0; q0 < cnt; q0 += 4) {
+      int es[4];
 #pragma unroll
-      for (int r = 0; r < BFMOE_MAX_K; ++r) {
-        if (r < k && df_ranks_before(ch, cl, ci, vh[r], vl[r], id[r])) {
-          const float th = vh[r], tl = vl[r];
-          const int ti = id[r];
-          vh[r] = ch;
-          vl[r] = cl;
-          id[r] = ci;
-          ch = th;
-          cl = tl;
-          ci = ti;
+      for (int j = 0; j < 4; ++j) es[j] = q0 + j < cnt ? (all ? q0 + j : win_s[w][q0 + j]) : -1;
+      float h4[4], l4[4];
+      df_logits4(xr, wg, bias, d, es, lane, h4, l4);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (es[j] < 0) break;
+        // every lane holds the same value: a uniform insertion
+        float ch = h4[j], cl = l4[j];
+        int ci = es[j];
+#pragma unroll
+        for (int r = 0; r < BFMOE_MAX_K; ++r) {
+          if (r < k && df_ranks_before(ch, cl, ci, vh[r], vl[r], id[r])) {
+            const float th = vh[r], tl = vl[r];
+            const int ti = id[r];
+            vh[r] = ch;
+            vl[r] = cl;
+            id[r] = ci;
+            ch = th;
+            cl = tl;
+            ci = ti;
+          }
         }
       }
     }
