@@ -340,6 +340,13 @@ def run_ours(args, wl):
         total_ms = timed(args.steps, graph.replay)
     launches = launches_per_step * args.steps
     torch.cuda.synchronize()
+    # sustained window: >= 1 s of timed graph replays (L2 flushed between
+    # them, outside the timed intervals), with its own clock samples
+    step_s = max(1e-6, total_ms / args.steps / 1e3)
+    sus_n = max(args.steps, int(math.ceil(1.0 / step_s)))
+    with ClockSampler(physical_gpu_index(local)) as sus_clocks:
+        sus_ms = timed(sus_n, graph.replay)
+    sus_ms = max_over_ranks(sus_ms)
     eager_ms = timed(args.steps, step)
     if world > 1:
         dist.barrier()
@@ -374,6 +381,27 @@ def run_ours(args, wl):
     e2e_eager_ms = max_over_ranks(e2e_eager_ms)
     B.bfmoe_check_device_error()
 
+    # --- decode batches: router + the add-only forward, T = 64 -------------------
+    dec_T = min(64, wl.tokens)
+    dec = B.ButterflyMoE(layer, wg, bias, wl.k, dec_T, x.dtype)
+    xd = x[:dec_T].contiguous()
+    yd = torch.empty_like(xd)
+    for _ in range(max(3, args.warmup)):
+        dec.decode(xd, y=yd)
+    torch.cuda.synchronize()
+    dec_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(dec_graph):
+        dec.decode(xd, y=yd)
+    dec_graph.replay()
+    torch.cuda.synchronize()
+    dec_steps = 200
+    dec_ms = timed(dec_steps, dec_graph.replay, flush_l2=False)
+    B.bfmoe_profile_enable(True)
+    timed(20, lambda: dec.decode(xd, y=yd), flush_l2=False)
+    dkt = B.bfmoe_profile_collect()
+    B.bfmoe_profile_enable(False)
+    B.bfmoe_check_device_error()
+
     if rank == 0:
         clk = clocks.summary()
         T = wl.tokens
@@ -393,6 +421,20 @@ def run_ours(args, wl):
         # its peak is then the sustained GEMM figure, else the burst one
         long_step = total_ms / args.steps > 1.0
         roof = roofline_entry(dom, kt[dom], costs, peaks, clk, workload=wl.name, sustained=long_step)
+        roof["algorithmic"] = ("2 R d^2 flops of the ternary product (R = T k routed rows); the fused "
+                               "kernel's inputs and outputs are the path's own bytes") \
+            if roof["bound"] == "tensor" else "bytes of the kernel's inputs and outputs"
+        if dom == "fused_expert":
+            # the same kernel seen from its CUDA-core work: two butterflies of
+            # L stages of d/2 rotations (4 multiplies, 2 adds) per routed row
+            rot_flops = 6.0 * T * wl.k * wl.d * L
+            avg_s = kt[dom][1] / kt[dom][0] / 1e3
+            fp32_peak = alu_peak_tflops(clk.get("sm_mhz") or 1965.0)
+            roof["rotation_view"] = {"bound": "alu", "flops_per_launch": rot_flops,
+                                     "achieved": rot_flops / avg_s / 1e12, "peak": fp32_peak, "unit": "TFLOP/s",
+                                     "frac": rot_flops / avg_s / 1e12 / fp32_peak,
+                                     "peak_source": "fp32 FMA lanes x 2 x median SM clock under load"}
+        as_built = as_built_bytes(wl)
         flops = 2.0 * T * wl.k * wl.d ** 2
         bytes_alg = algorithmic_bytes(wl)
         t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_alg / (peaks["hbm_gbs"] * 1e9))
@@ -402,6 +444,7 @@ def run_ours(args, wl):
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": workload_config(wl, "flushed between steps (512 MiB write, outside the timed intervals)"),
             "roofline": roof,
+            "as_built_traffic": as_built,
             "path_roofline": {"time_us": t_roof * 1e6, "achieved_us": 1e3 * total_ms / args.steps,
                               "frac": t_roof / (total_ms / args.steps / 1e3),
                               "formula": "max(2 T k d^2 / bf16 peak, algorithmic bytes / HBM BW)",
@@ -419,16 +462,46 @@ def run_ours(args, wl):
                             "captured once as a CUDA graph and replayed per step",
                     "eager_value": T * world * args.steps / (e2e_eager_ms / 1e3)},
             "gpu_launches": int(launches),
+            "sustained": {"steps": sus_n, "timed_seconds": sus_ms / 1e3, "ms_per_step": sus_ms / sus_n,
+                          "value": T * world * sus_n / (sus_ms / 1e3), "clocks": sus_clocks.summary()},
+            "decode": {"tokens": dec_T, "call": "router (bfmoe_router_topk) + bfmoe_decode_forward (add-only "
+                       "ternary product, float32 inside), CUDA-graph replays, weights L2-resident",
+                       "us_per_step": 1e3 * dec_ms / dec_steps,
+                       "tokens_per_s": dec_T * dec_steps / (dec_ms / 1e3),
+                       "kernels_us": {n: 1e3 * ms / c for n, (c, ms) in dkt.items()}},
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(inp, args.cpu_fraction)
         print(json.dumps(line), flush=True)
-    del graph, host_graph
+    del graph, host_graph, dec_graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def as_built_bytes(wl):
+    """Memory traffic the built pipeline adds per step on top of the
+    algorithmic bytes (not counted in any roofline fraction)."""
+    d, N, k, T = wl.d, wl.n_experts, wl.k, wl.tokens
+    L = wl.stages
+    R = T * k
+    xb = 2 if wl.dtype == "bf16" else 4
+    fused = wl.dtype == "bf16" and 64 <= d <= 512
+    out = {
+        "router_logits_f32": T * N * 4,                     # written for the fix-up of undecided tokens
+        "router_weight_split_bf16": 3 * N * d * 2,          # written, then read by the tensor-core router
+        "x_gather_rereads": (k - 1) * T * d * xb,           # each token's row is read once per slot
+        "weight_tables": 2 * N * L * (d // 2) * 8 * 2,      # cos/sin quads written and read per step
+        "base_bf16_copy": 2 * d * d * 2,                    # the expanded base, written and read
+        "slot_buffer": 2 * R * d * (2 if fused else 4),     # gated rows written, then summed by the combine
+    }
+    if not fused:
+        out["x_rot_round_trip"] = 2 * R * d * (2 if wl.dtype == "bf16" else 4)
+        out["z_round_trip"] = 2 * R * d * (2 if wl.dtype == "bf16" else 4)
+    out["total"] = sum(out.values())
+    return out
 
 
 def algorithmic_bytes(wl):
@@ -449,41 +522,29 @@ NCU_KERNEL = {"fused_expert": "fused_expert_kernel", "post_rotate": "post_rotate
 
 
 def kernel_sources_hash() -> str:
-    """sha256 over the library's CUDA sources (sorted by name)."""
-    import hashlib
-    d = os.path.join(ROOT, "ternary_butterfly_experts_b200", "csrc")
-    h = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(f.encode())
-            with open(os.path.join(d, f), "rb") as fh:
-                h.update(fh.read())
-    return h.hexdigest()
+    """sha256 over the library's CUDA sources under ROOT (sorted by name)."""
+    from ternary_butterfly_experts_b200.ncu_summary import kernel_sources_hash as h
+    return h(os.path.join(ROOT, "ternary_butterfly_experts_b200", "csrc"))
 
 
 def profiled_traffic(name, workload):
-    """DRAM bytes (read + write) of one launch of kernel `name` from the
-    committed ncu summary of this workload, or None when there is none or the
-    kernel sources have changed since it was taken."""
+    """DRAM bytes (read + write) of one launch of kernel `name`, from the
+    committed ncu summary (profiles/ncu_*_<workload>.json, written by
+    ternary_butterfly_experts_b200.ncu_summary), or None when there is none or
+    the kernel sources have changed since it was taken."""
     import glob
-    import re
     kname = NCU_KERNEL.get(name)
     if kname is None:
         return None
     src_hash = kernel_sources_hash()
-    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"ncu_full_*_{workload}.md"))):
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"ncu_*_{workload}.json"))):
         with open(path) as f:
-            text = f.read()
-        m = re.search(r"kernel sources sha256: ([0-9a-f]{64})", text)
-        if not m or m.group(1) != src_hash:
+            js = json.load(f)
+        if js.get("kernel_sources_sha256") != src_hash:
             continue
-        sec = re.search(r"## `" + re.escape(kname) + r"[^`]*`(.*?)(?=\n## |\Z)", text, re.S)
-        if not sec:
-            continue
-        rd = re.search(r"dram__bytes_read\.sum \| ([0-9.]+) Mbyte", sec.group(1))
-        wr = re.search(r"dram__bytes_write\.sum \| ([0-9.]+) Mbyte", sec.group(1))
-        if rd and wr:
-            return (float(rd.group(1)) + float(wr.group(1))) * 1e6
+        for kn, e in js.get("kernels", {}).items():
+            if kn.split("<")[0] == kname and "dram_bytes_per_launch" in e:
+                return float(e["dram_bytes_per_launch"])
     return None
 
 
@@ -512,7 +573,8 @@ def roofline_entry(name, kt_entry, costs, peaks, clk, workload=None, sustained=F
     return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak, "traffic": traffic, "avg_launch_us": avg_s * 1e6,
             "work_per_launch": work, "peak_source": src,
-            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, first launch (profiles/)"
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, first launch "
+                              "(profiles/ncu_*.json of the current kernel sources)"
             if traffic is not None else "no ncu summary taken from the current kernel sources"}
 
 

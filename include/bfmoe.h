@@ -289,6 +289,29 @@ int bfmoe_backward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, 
 size_t bfmoe_backward_workspace_size(int d, int n_experts, int T, int k);
 
 /*
+ * Add-only expert forward for small batches (decode).  The ternary product
+ * of each expert is a signed sum of its inputs (technical summary, 2.3 step
+ * 2): this call computes
+ *   y_t = sum_j gates[t][j] * B(phi_e) (alpha * W_base (B(theta_e)^T x_t)),
+ *   e = idx[t][j], j ascending,
+ * decoding the 2-bit codes of W_base in registers and adding, subtracting or
+ * skipping each rotated input (no multiplications in the product), with every
+ * intermediate in float32 and one rounding of y to x_dtype.  One CTA per
+ * token: meant for decode batches (T up to a few hundred), correct for any
+ * T >= 0.
+ *   layer     as for bfmoe_forward (the prepared tables are not used)
+ *   x         device [T][d], dtype x_dtype
+ *   idx, gates device [T][k] as written by bfmoe_router_topk (the bucket
+ *             arrays are not needed)
+ *   y         device [T][d], dtype x_dtype (written)
+ * No workspace.  Returns BFMOE_EINVAL on bad arguments (nothing launched);
+ * an expert id outside [0, N) is skipped and recorded as
+ * BFMOE_EDEVICE_BOUNDS in the device error word.
+ */
+int bfmoe_decode_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, int k,
+                         const int32_t* idx, const float* gates, void* y, bfmoe_stream_t stream);
+
+/*
  * Form expert e densely, alpha * B(phi_e) . W_base . B(theta_e)^T, in float32
  * (technical summary, 2.1).  For checking only.
  *   w_out     device float [d][d] (written), row = output

@@ -23,7 +23,7 @@ __all__ = [
     "BfmoeError", "Layer", "ButterflyMoE", "bfmoe_pack_base", "bfmoe_unpack_base", "bfmoe_router_topk",
     "bfmoe_router_topk_noalloc", "bfmoe_moe_forward", "bfmoe_moe_workspace_size", "bfmoe_prepare_layer",
     "bfmoe_layer_tables_size", "bfmoe_backward", "bfmoe_backward_workspace_size",
-    "bfmoe_forward", "bfmoe_materialize_expert", "bfmoe_workspace_size", "bfmoe_router_scratch_size", "bfmoe_check_device_error",
+    "bfmoe_forward", "bfmoe_decode_forward", "bfmoe_materialize_expert", "bfmoe_workspace_size", "bfmoe_router_scratch_size", "bfmoe_check_device_error",
     "bfmoe_launch_count", "bfmoe_profile_enable", "bfmoe_profile_collect", "bfmoe_last_error", "workspace",
 ]
 
@@ -240,6 +240,23 @@ def bfmoe_forward(layer: Layer, x, k: int, idx, gates, offsets, rows, ws, y=None
     return y
 
 
+def bfmoe_decode_forward(layer: Layer, x, k: int, idx, gates, y=None, stream=None):
+    """Add-only small-batch forward: y [T][d] (dtype of x) from the routing
+    idx / gates, the ternary product done by signed sums, float32 inside."""
+    torch = _torch()
+    _need(x, "x")
+    T, d = x.shape
+    if d != layer.d:
+        raise ValueError(f"x has width {d}, layer has d={layer.d}")
+    _need(idx, "idx", torch.int32)
+    _need(gates, "gates", torch.float32)
+    if y is None:
+        y = torch.empty_like(x)
+    capi.check(capi.lib().bfmoe_decode_forward(
+        ctypes.byref(layer.c), _ptr(x), _dtype_code(x), T, k, _ptr(idx), _ptr(gates), _ptr(y), _stream(stream)))
+    return y
+
+
 def bfmoe_backward_workspace_size(d: int, n_experts: int, T: int, k: int) -> int:
     return int(capi.lib().bfmoe_backward_workspace_size(d, n_experts, T, k))
 
@@ -400,6 +417,16 @@ class ButterflyMoE:
         y, _ = bfmoe_moe_forward(self.layer, x, self.w_gate, self.bias, self.k, self.ws_moe, routing=routing, y=y,
                                  stream=stream)
         return y
+
+    def decode(self, x, y=None, stream=None):
+        """Router + the add-only small-batch forward (bfmoe_decode_forward)."""
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError("more tokens than the buffers hold")
+        if y is None:
+            y = self.y_dev[:T]
+        idx, gates, _, _, _ = self.route(x, stream=stream)
+        return bfmoe_decode_forward(self.layer, x, self.k, idx, gates, y=y, stream=stream)
 
     def forward_host(self, x_host, y_host, chunk: int = 0, stream=None):
         """The end-to-end call: pinned host tokens in, pinned host outputs back,

@@ -68,6 +68,7 @@ SIGNATURES = {
     "bfmoe_moe_forward_host": (_I, [ctypes.POINTER(BfmoeLayer), _P, _I, _I, _P, _P, _I, _P, _I, _P, _SZ, _P]),
     "bfmoe_moe_host_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "bfmoe_materialize_expert": (_I, [ctypes.POINTER(BfmoeLayer), _I, _P, _P]),
+    "bfmoe_decode_forward": (_I, [ctypes.POINTER(BfmoeLayer), _P, _I, _I, _I, _P, _P, _P, _P]),
     "bfmoe_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "bfmoe_router_scratch_size": (_SZ, [_I, _I, _I, _I, _I]),
     "bfmoe_last_error": (ctypes.c_char_p, []),

@@ -16,6 +16,7 @@
 #include "backward.cuh"
 #include "bucket.cuh"
 #include "common.cuh"
+#include "decode.cuh"
 #include "fused_tc.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
@@ -1129,6 +1130,39 @@ int bfmoe_router_topk_noalloc(const void* x, int x_dtype, int T, int d, const fl
   if ((rc = noalloc_scratch(&scratch))) return rc;
   return bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, n_experts, k, idx, gates, counts, offsets, rows, scratch,
                            BFMOE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+int bfmoe_decode_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, int k, const int32_t* idx,
+                         const float* gates, void* y, bfmoe_stream_t stream) {
+  if (!layer) return fail(BFMOE_EINVAL, "decode_forward: NULL layer");
+  int rc = check_sizes(layer->d, layer->n_experts, T, k);
+  if (rc) return rc;
+  if ((rc = check_dtype(x_dtype))) return rc;
+  if (T == 0) return ok();
+  if (!layer->w_packed || !layer->theta || !layer->phi) return fail(BFMOE_EINVAL, "decode_forward: NULL layer weights");
+  if (!x || !idx || !gates || !y) return fail(BFMOE_EINVAL, "decode_forward: NULL pointer");
+  const int d = layer->d, L = ilog2(d), N = layer->n_experts;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t smem = static_cast<size_t>(2) * decode_rows(d, k) * d * sizeof(float);  // <= 128 KiB
+  static std::atomic<uint64_t> done{0};
+  if (needs_attr(done)) {
+    const int most = 2 * 16384 * static_cast<int>(sizeof(float));
+    cudaFuncSetAttribute(decode_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    cudaFuncSetAttribute(decode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    attr_set(done);
+  }
+  const int grid = grid_for(T, 1, sm_count() * 8);
+  const cudaError_t e = launch("decode", s, [&] {
+    if (x_dtype == BFMOE_BF16)
+      pdl_launch(decode_kernel<__nv_bfloat16>, grid, kDecodeThreads, smem, s, static_cast<const __nv_bfloat16*>(x),
+                 T, d, L, k, idx, gates, layer->w_packed, layer->alpha, layer->theta, layer->phi, N,
+                 static_cast<__nv_bfloat16*>(y));
+    else
+      pdl_launch(decode_kernel<float>, grid, kDecodeThreads, smem, s, static_cast<const float*>(x), T, d, L, k, idx,
+                 gates, layer->w_packed, layer->alpha, layer->theta, layer->phi, N, static_cast<float*>(y));
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "decode_forward");
+  return ok();
 }
 
 int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, int k, const int32_t* idx,

@@ -51,11 +51,10 @@ def test_roofline_peak_choice():
 
 
 def _summary(src_hash):
-    return (f"# ncu --set full\n\nkernel sources sha256: {src_hash}\n\n"
-            "## `post_rotate_fast_kernel<16, __nv_bfloat16, __nv_bfloat16>`\n\n| metric | value |\n|---|---|\n"
-            "| dram__bytes_read.sum | 38.5 Mbyte |\n| dram__bytes_write.sum | 1.5 Mbyte |\n\n"
-            "## `pre_rotate_fast_kernel<16, __nv_bfloat16, __nv_bfloat16>`\n\n| metric | value |\n|---|---|\n"
-            "| dram__bytes_read.sum | 20.0 Mbyte |\n| dram__bytes_write.sum | 2.0 Mbyte |\n")
+    return {"kind": "ncu --set full", "workload": "d512_n256", "command": "ncu ...",
+            "kernel_sources_sha256": src_hash,
+            "kernels": {"fused_expert_kernel<512>": {"dram_bytes_per_launch": 27.9e6},
+                        "router_tc_kernel<128, 3, 2>": {"dram_bytes_per_launch": 17.6e6}}}
 
 
 @pytest.fixture
@@ -69,14 +68,15 @@ def fake_root(tmp_path, monkeypatch):
 
 
 def test_traffic_read_only_for_the_current_sources(fake_root):
-    path = fake_root / "profiles" / "ncu_full_rotations_d512_n256.md"
-    path.write_text(_summary(bench.kernel_sources_hash()))
-    assert bench.profiled_traffic("post_rotate", "d512_n256") == pytest.approx(40.0e6)
-    assert bench.profiled_traffic("pre_rotate", "d512_n256") == pytest.approx(22.0e6)
+    import json
+    path = fake_root / "profiles" / "ncu_fused_expert_d512_n256.json"
+    path.write_text(json.dumps(_summary(bench.kernel_sources_hash())))
+    assert bench.profiled_traffic("fused_expert", "d512_n256") == pytest.approx(27.9e6)
+    assert bench.profiled_traffic("router_tc", "d512_n256") == pytest.approx(17.6e6)
     assert bench.profiled_traffic("combine", "d512_n256") is None          # not in the summary
-    assert bench.profiled_traffic("post_rotate", "d1024_n256") is None     # another workload
-    path.write_text(_summary("0" * 64))                                     # taken from other sources
-    assert bench.profiled_traffic("post_rotate", "d512_n256") is None
+    assert bench.profiled_traffic("fused_expert", "d1024_n256") is None    # another workload
+    path.write_text(json.dumps(_summary("0" * 64)))                         # taken from other sources
+    assert bench.profiled_traffic("fused_expert", "d512_n256") is None
 
 
 def test_source_hash_follows_the_sources(fake_root):
@@ -84,3 +84,15 @@ def test_source_hash_follows_the_sources(fake_root):
     with open(fake_root / "ternary_butterfly_experts_b200" / "csrc" / "combine_probe.cuh", "w") as f:
         f.write("// a new source file\n")
     assert bench.kernel_sources_hash() != before
+
+
+def test_as_built_traffic_is_listed_apart():
+    wl = W.WORKLOADS["d512_n256"]
+    ab = bench.as_built_bytes(wl)
+    # the fused path keeps X_rot and Z on chip; the slot buffer and the logits remain
+    assert "x_rot_round_trip" not in ab and "z_round_trip" not in ab
+    assert ab["slot_buffer"] == 2 * 32768 * 512 * 2
+    assert ab["router_logits_f32"] == 16384 * 256 * 4
+    assert ab["total"] == sum(v for k, v in ab.items() if k != "total")
+    ab4 = bench.as_built_bytes(W.WORKLOADS["d2048_n1024"])
+    assert ab4["x_rot_round_trip"] == 2 * 131072 * 4 * 2048 * 2
