@@ -464,7 +464,7 @@ def run_ours(args, wl):
             "gpu_launches": int(launches),
             "sustained": {"steps": sus_n, "timed_seconds": sus_ms / 1e3, "ms_per_step": sus_ms / sus_n,
                           "value": T * world * sus_n / (sus_ms / 1e3), "clocks": sus_clocks.summary()},
-            "decode": {"tokens": dec_T, "call": "router (bfmoe_router_topk) + bfmoe_decode_forward (add-only "
+            "decode": {"tokens": dec_T, "call": "router (bfmoe_router_topk, no buckets) + bfmoe_decode_forward (add-only "
                        "ternary product, float32 inside), CUDA-graph replays, weights L2-resident",
                        "us_per_step": 1e3 * dec_ms / dec_steps,
                        "tokens_per_s": dec_T * dec_steps / (dec_ms / 1e3),

@@ -114,7 +114,10 @@ int bfmoe_unpack_base(const uint32_t* w_packed, int d, uint16_t* w_bf16, bfmoe_s
  *             routed rows r = t*k + j in ascending token order
  *   ws        device scratch of at least bfmoe_workspace_size(...) bytes,
  *             256-byte aligned
- * T = 0 is allowed (counts and offsets are zeroed).
+ * counts, offsets and rows may all three be NULL: the buckets are then not
+ * built (bfmoe_decode_forward needs only idx and gates).  One or two of them
+ * NULL is BFMOE_EINVAL.
+ * T = 0 is allowed (counts and offsets, when given, are zeroed).
  */
 int bfmoe_router_topk(const void* x, int x_dtype, int T, int d,
                       const float* w_gate, const float* bias, int n_experts, int k,

@@ -116,8 +116,9 @@ def bfmoe_unpack_base(w_packed, d: int, out=None, stream=None):
     return out
 
 
-def bfmoe_router_topk(x, w_gate, bias, k: int, ws, out=None, stream=None):
-    """Returns (idx [T,k] int32, gates [T,k] f32, counts [N], offsets [N+1], rows [T*k])."""
+def bfmoe_router_topk(x, w_gate, bias, k: int, ws, out=None, stream=None, buckets: bool = True):
+    """Returns (idx [T,k] int32, gates [T,k] f32, counts [N], offsets [N+1], rows [T*k]);
+    with ``buckets=False`` the last three are None and are not built."""
     torch = _torch()
     _need(x, "x")
     _need(w_gate, "w_gate", torch.float32)
@@ -128,10 +129,10 @@ def bfmoe_router_topk(x, w_gate, bias, k: int, ws, out=None, stream=None):
     dev = x.device
     if out is None:
         out = (torch.empty((T, k), dtype=torch.int32, device=dev),
-               torch.empty((T, k), dtype=torch.float32, device=dev),
-               torch.empty((N,), dtype=torch.int32, device=dev),
-               torch.empty((N + 1,), dtype=torch.int32, device=dev),
-               torch.empty((T * k,), dtype=torch.int32, device=dev))
+               torch.empty((T, k), dtype=torch.float32, device=dev))
+        out += (torch.empty((N,), dtype=torch.int32, device=dev),
+                torch.empty((N + 1,), dtype=torch.int32, device=dev),
+                torch.empty((T * k,), dtype=torch.int32, device=dev)) if buckets else (None, None, None)
     idx, gates, counts, offsets, rows = out
     capi.check(capi.lib().bfmoe_router_topk(
         _ptr(x), _dtype_code(x), T, d, _ptr(w_gate), _ptr(bias), N, k, _ptr(idx), _ptr(gates),
@@ -419,13 +420,16 @@ class ButterflyMoE:
         return y
 
     def decode(self, x, y=None, stream=None):
-        """Router + the add-only small-batch forward (bfmoe_decode_forward)."""
+        """Router (no buckets) + the add-only small-batch forward
+        (bfmoe_decode_forward)."""
         T = x.shape[0]
         if T > self.max_tokens:
             raise ValueError("more tokens than the buffers hold")
         if y is None:
             y = self.y_dev[:T]
-        idx, gates, _, _, _ = self.route(x, stream=stream)
+        idx, gates = self.idx[:T], self.gates[:T]
+        bfmoe_router_topk(x, self.w_gate, self.bias, self.k, self.ws, out=(idx, gates, None, None, None),
+                          stream=stream)
         return bfmoe_decode_forward(self.layer, x, self.k, idx, gates, y=y, stream=stream)
 
     def forward_host(self, x_host, y_host, chunk: int = 0, stream=None):

@@ -1007,15 +1007,19 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
   int rc = check_sizes(d, n_experts, T, k);
   if (rc) return rc;
   if ((rc = check_dtype(x_dtype))) return rc;
-  if (!counts || !offsets) return fail(BFMOE_EINVAL, "router_topk: NULL counts/offsets");
+  // the buckets are built when all three outputs are given, skipped when none is
+  const bool buckets = counts || offsets || rows;
+  if (buckets && (!counts || !offsets || !rows))
+    return fail(BFMOE_EINVAL, "router_topk: counts, offsets and rows must be all given or all NULL");
   const int N = n_experts;
   cudaError_t e;
   if (T == 0) {
+    if (!buckets) return ok();
     if ((e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * N, s)) != cudaSuccess) return cuda_fail(e, "router_topk: memset");
     if ((e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (N + 1), s)) != cudaSuccess) return cuda_fail(e, "router_topk: memset");
     return ok();
   }
-  if (!x || !w_gate || !idx || !gates || !rows) return fail(BFMOE_EINVAL, "router_topk: NULL pointer");
+  if (!x || !w_gate || !idx || !gates) return fail(BFMOE_EINVAL, "router_topk: NULL pointer");
   const Plan p = make_plan(d, N, T, k, x_dtype);
   if ((rc = check_ws(p, ws, ws_bytes, p.rt_end))) return rc;
   uint8_t* W = static_cast<uint8_t*>(ws);
@@ -1090,6 +1094,7 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
   }
 
   const int chunk = bucket_chunk(k);
+  if (!buckets) return ok();
   const int nchunks = static_cast<int>((R + chunk - 1) / chunk);
   static std::atomic<uint64_t> done{0};
   if (needs_attr(done)) {

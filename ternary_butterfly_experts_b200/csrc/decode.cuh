@@ -22,7 +22,7 @@
 
 namespace bfmoe {
 
-constexpr int kDecodeThreads = 256;
+constexpr int kDecodeThreads = 512;
 constexpr int kDecodeRows = 8;                                  // slots of a token handled together
 constexpr int kDecodeOut = BFMOE_MAX_D / kDecodeThreads;        // outputs per thread, at most
 
@@ -59,6 +59,50 @@ __device__ __forceinline__ void decode_stage(float* v, const float* const* ang, 
     }
   }
   __syncthreads();
+}
+
+// z[j][o] = alpha * sum_i W_base[o][i] u[j][i] for the NJ rows of u, one
+// output o per thread at a time: the 16 codes of a word are decoded from a
+// register and each adds u_i to the row's positive or negative sum, or
+// nothing.  Rows are d floats apart in shared memory.
+template <int NJ>
+__device__ __forceinline__ void decode_product(const float* u, float* z, const uint32_t* __restrict__ w_packed, int d,
+                                               int words, float alpha) {
+  for (int o = threadIdx.x; o < d; o += blockDim.x) {
+    const uint32_t* wr = w_packed + static_cast<size_t>(o) * words;
+    float pos[NJ], neg[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) pos[j] = neg[j] = 0.f;
+    if (d >= 16) {
+#pragma unroll 2
+      for (int w = 0; w < words; ++w) {
+        const uint32_t word = __ldg(wr + w);
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+          const uint32_t c = (word >> (2 * b)) & 3u;
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) {
+            const float ui = u[static_cast<size_t>(j) * d + 16 * w + b];
+            pos[j] += c == 1u ? ui : 0.f;
+            neg[j] += c == 3u ? ui : 0.f;
+          }
+        }
+      }
+    } else {
+      const uint32_t word = __ldg(wr);  // one word holds the whole row
+      for (int b = 0; b < d; ++b) {
+        const uint32_t c = (word >> (2 * b)) & 3u;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const float ui = u[static_cast<size_t>(j) * d + b];
+          pos[j] += c == 1u ? ui : 0.f;
+          neg[j] += c == 3u ? ui : 0.f;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) z[static_cast<size_t>(j) * d + o] = alpha * (pos[j] - neg[j]);
+  }
 }
 
 template <typename Tx>
@@ -101,33 +145,15 @@ __global__ __launch_bounds__(kDecodeThreads) void decode_kernel(const Tx* __rest
       for (int s = L - 1; s >= 0; --s) decode_stage<true>(u, th_s, nj, d, s);
       // the ternary product of every slot row at once: each 2-bit code adds
       // u_i, subtracts it or skips it; a row's code words are loaded once
-      for (int o = threadIdx.x; o < d; o += blockDim.x) {
-        const uint32_t* wr = w_packed + static_cast<size_t>(o) * words;
-        float pos[kDecodeRows], neg[kDecodeRows];
-#pragma unroll
-        for (int jj = 0; jj < kDecodeRows; ++jj) pos[jj] = neg[jj] = 0.f;
-#pragma unroll 4
-        for (int w = 0; w < words; ++w) {
-          const uint32_t word = wr[w];
-          const int n = d - 16 * w < 16 ? d - 16 * w : 16;
-#pragma unroll
-          for (int b = 0; b < 16; ++b) {
-            if (b < n) {
-              const uint32_t c = (word >> (2 * b)) & 3u;
-#pragma unroll
-              for (int jj = 0; jj < kDecodeRows; ++jj) {
-                if (jj < nj) {
-                  const float ui = u[static_cast<size_t>(jj) * d + 16 * w + b];
-                  pos[jj] += c == 1u ? ui : 0.f;
-                  neg[jj] += c == 3u ? ui : 0.f;
-                }
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int jj = 0; jj < kDecodeRows; ++jj)
-          if (jj < nj) z[static_cast<size_t>(jj) * d + o] = alpha * (pos[jj] - neg[jj]);
+      switch (nj) {
+        case 1: decode_product<1>(u, z, w_packed, d, words, alpha); break;
+        case 2: decode_product<2>(u, z, w_packed, d, words, alpha); break;
+        case 3: decode_product<3>(u, z, w_packed, d, words, alpha); break;
+        case 4: decode_product<4>(u, z, w_packed, d, words, alpha); break;
+        case 5: decode_product<5>(u, z, w_packed, d, words, alpha); break;
+        case 6: decode_product<6>(u, z, w_packed, d, words, alpha); break;
+        case 7: decode_product<7>(u, z, w_packed, d, words, alpha); break;
+        default: decode_product<8>(u, z, w_packed, d, words, alpha); break;
       }
       __syncthreads();
       for (int s = 0; s < L; ++s) decode_stage<false>(z, ph_s, nj, d, s);

@@ -89,3 +89,14 @@ def test_host_workspace_size(L):
     assert L.bfmoe_moe_host_workspace_size(512, 256, 16384, 2, bf, 16384) > full  # one big chunk needs more
     assert L.bfmoe_moe_host_workspace_size(500, 256, 16384, 2, bf, 0) == 0
     assert L.bfmoe_moe_host_workspace_size(512, 4, 100, 5, bf, 0) == 0
+
+
+def test_router_rejects_partial_bucket_outputs():
+    """counts, offsets and rows: all given or all NULL (checked before any launch)."""
+    import ctypes
+    L = capi.lib()
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    rc = L.bfmoe_router_topk(p, 1, 0, 64, p, None, 4, 2, p, p, p, None, None, p, 64, None)
+    assert rc == 1  # BFMOE_EINVAL
+    assert b"all given or all NULL" in L.bfmoe_last_error()

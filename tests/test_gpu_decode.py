@@ -115,3 +115,16 @@ def test_decode_out_of_range_expert_is_reported():
     with pytest.raises(B().BfmoeError):
         B().bfmoe_check_device_error()
     B().bfmoe_check_device_error()  # the word is cleared by the read
+
+
+def test_router_without_buckets_matches_with_buckets():
+    """counts / offsets / rows all NULL: the same idx and gates, no buckets."""
+    inp = W.generate(W.WORKLOADS["d512_n256"], seed=3, tokens=64)
+    x = inp.x.cuda().contiguous()
+    wg = torch.from_numpy(inp.w_gate).cuda()
+    bias = torch.from_numpy(inp.bias).cuda()
+    ws = B().workspace(512, 256, 64, 2, B().BFMOE_BF16)
+    i1, g1, c1, _, _ = B().bfmoe_router_topk(x, wg, bias, 2, ws)
+    i2, g2, c2, o2, r2 = B().bfmoe_router_topk(x, wg, bias, 2, ws, buckets=False)
+    assert c2 is None and o2 is None and r2 is None
+    assert torch.equal(i1, i2) and torch.equal(g1, g2)
