@@ -402,6 +402,25 @@ def run_ours(args, wl):
     B.bfmoe_profile_enable(False)
     B.bfmoe_check_device_error()
 
+    # --- backward: dx, both angle sets, the base (straight-through), alpha, W_g, b
+    routing = (model.idx[:wl.tokens], model.gates[:wl.tokens], model.counts, model.offsets,
+               model.rows[:wl.tokens * wl.k])
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    gy = torch.randn(x.shape, dtype=torch.float32, device=dev, generator=g)
+    bw_ws = torch.empty(max(B.bfmoe_backward_workspace_size(wl.d, wl.n_experts, wl.tokens, wl.k), 256),
+                        dtype=torch.uint8, device=dev)
+
+    def backward():
+        B.bfmoe_backward(layer, x, wl.k, wg, routing, gy, bias_grad=bias is not None, ws=bw_ws)
+
+    for _ in range(2):
+        backward()
+    torch.cuda.synchronize()
+    bw_steps = 3
+    bw_ms = timed(bw_steps, backward)
+    B.bfmoe_check_device_error()
+
     if rank == 0:
         clk = clocks.summary()
         T = wl.tokens
@@ -464,6 +483,9 @@ def run_ours(args, wl):
             "gpu_launches": int(launches),
             "sustained": {"steps": sus_n, "timed_seconds": sus_ms / 1e3, "ms_per_step": sus_ms / sus_n,
                           "value": T * world * sus_n / (sus_ms / 1e3), "clocks": sus_clocks.summary()},
+            "backward": {"call": "bfmoe_backward (dx, dtheta, dphi, straight-through dW_base, dalpha, dW_g, db) "
+                                 "on the step's routing, eager, L2 flushed", "steps": bw_steps,
+                         "ms_per_step": bw_ms / bw_steps, "tokens_per_s": T * bw_steps / (bw_ms / 1e3)},
             "decode": {"tokens": dec_T, "call": "router (bfmoe_router_topk, no buckets) + bfmoe_decode_forward (add-only "
                        "ternary product, float32 inside), CUDA-graph replays, weights L2-resident",
                        "us_per_step": 1e3 * dec_ms / dec_steps,

@@ -115,8 +115,8 @@ int bfmoe_unpack_base(const uint32_t* w_packed, int d, uint16_t* w_bf16, bfmoe_s
  *   ws        device scratch of at least bfmoe_workspace_size(...) bytes,
  *             256-byte aligned
  * counts, offsets and rows may all three be NULL: the buckets are then not
- * built (bfmoe_decode_forward needs only idx and gates).  One or two of them
- * NULL is BFMOE_EINVAL.
+ * built (bfmoe_decode_forward needs only idx and gates).  Otherwise counts
+ * and offsets, and rows when T > 0, must all be given (else BFMOE_EINVAL).
  * T = 0 is allowed (counts and offsets, when given, are zeroed).
  */
 int bfmoe_router_topk(const void* x, int x_dtype, int T, int d,

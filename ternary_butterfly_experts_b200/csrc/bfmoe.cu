@@ -1007,9 +1007,10 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
   int rc = check_sizes(d, n_experts, T, k);
   if (rc) return rc;
   if ((rc = check_dtype(x_dtype))) return rc;
-  // the buckets are built when all three outputs are given, skipped when none is
+  // the buckets are built when counts and offsets are given (rows too, unless
+  // T = 0), skipped when all three are NULL
   const bool buckets = counts || offsets || rows;
-  if (buckets && (!counts || !offsets || !rows))
+  if (buckets && (!counts || !offsets || (!rows && T > 0)))
     return fail(BFMOE_EINVAL, "router_topk: counts, offsets and rows must be all given or all NULL");
   const int N = n_experts;
   cudaError_t e;
