@@ -456,8 +456,8 @@ cudaError_t launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const C
 
 template <int BN, int STAGES, int K>
 cudaError_t launch_router_tc_k(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
-                               float eps_c, float* logits, int* unsure, int32_t* idx, float* gates,
-                               int32_t* cc, cudaStream_t s) {
+                               float eps_c, float* logits, const __nv_bfloat16* x, const float* w_gate,
+                               int32_t* idx, float* gates, int32_t* cc, cudaStream_t s) {
   using Cfg = RouterTcCfg<BN, STAGES>;
   static std::atomic<uint64_t> done{0};
   if (needs_attr(done)) {
@@ -469,23 +469,23 @@ cudaError_t launch_router_tc_k(const CUtensorMap& tx, const CUtensorMap& tw, con
   const int grid = (T + kGemmBM - 1) / kGemmBM;
   return launch("router_tc", s, [&] {
     pdl_launch(router_tc_kernel<BN, STAGES, K>, grid, kRouterThreads, Cfg::SMEM_BYTES, s, tx, tw, bias, T, d, N,
-               eps_c, logits, unsure, idx, gates, cc);
+               eps_c, logits, x, w_gate, idx, gates, cc);
   });
 }
 
 template <int BN, int STAGES>
 cudaError_t launch_router_tc(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias, int T, int d, int N,
-                             int k, float eps_c, float* logits, int* unsure, int32_t* idx, float* gates,
-                             int32_t* cc, cudaStream_t s) {
+                             int k, float eps_c, float* logits, const __nv_bfloat16* x, const float* w_gate,
+                             int32_t* idx, float* gates, int32_t* cc, cudaStream_t s) {
   switch (k) {
-    case 1: return launch_router_tc_k<BN, STAGES, 1>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
-    case 2: return launch_router_tc_k<BN, STAGES, 2>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
-    case 3: return launch_router_tc_k<BN, STAGES, 3>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
-    case 4: return launch_router_tc_k<BN, STAGES, 4>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
-    case 5: return launch_router_tc_k<BN, STAGES, 5>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
-    case 6: return launch_router_tc_k<BN, STAGES, 6>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
-    case 7: return launch_router_tc_k<BN, STAGES, 7>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
-    default: return launch_router_tc_k<BN, STAGES, 8>(tx, tw, bias, T, d, N, eps_c, logits, unsure, idx, gates, cc, s);
+    case 1: return launch_router_tc_k<BN, STAGES, 1>(tx, tw, bias, T, d, N, eps_c, logits, x, w_gate, idx, gates, cc, s);
+    case 2: return launch_router_tc_k<BN, STAGES, 2>(tx, tw, bias, T, d, N, eps_c, logits, x, w_gate, idx, gates, cc, s);
+    case 3: return launch_router_tc_k<BN, STAGES, 3>(tx, tw, bias, T, d, N, eps_c, logits, x, w_gate, idx, gates, cc, s);
+    case 4: return launch_router_tc_k<BN, STAGES, 4>(tx, tw, bias, T, d, N, eps_c, logits, x, w_gate, idx, gates, cc, s);
+    case 5: return launch_router_tc_k<BN, STAGES, 5>(tx, tw, bias, T, d, N, eps_c, logits, x, w_gate, idx, gates, cc, s);
+    case 6: return launch_router_tc_k<BN, STAGES, 6>(tx, tw, bias, T, d, N, eps_c, logits, x, w_gate, idx, gates, cc, s);
+    case 7: return launch_router_tc_k<BN, STAGES, 7>(tx, tw, bias, T, d, N, eps_c, logits, x, w_gate, idx, gates, cc, s);
+    default: return launch_router_tc_k<BN, STAGES, 8>(tx, tw, bias, T, d, N, eps_c, logits, x, w_gate, idx, gates, cc, s);
   }
 }
 
@@ -1031,9 +1031,8 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
   const long long R = static_cast<long long>(T) * k;
   // the float32 error band that leaves a top-k undecided (router.cuh)
   const float eps_c = 2e-5f * std::sqrt(static_cast<float>(d) / 2048.f);
-  if ((e = cudaMemsetAsync(unsure, 0, 8, s)) != cudaSuccess) return cuda_fail(e, "router_topk: memset");
-
   const bool tc_router = tc_router_path(x_dtype, d);
+  if (!tc_router && (e = cudaMemsetAsync(unsure, 0, 8, s)) != cudaSuccess) return cuda_fail(e, "router_topk: memset");
   if (tc_router) {
     // tensor cores: exact 3-way bf16 split of W_g, top-k fused in the epilogue
     if (!aligned16(x)) return fail(BFMOE_EINVAL, "router_topk: x must be 16-byte aligned");
@@ -1044,14 +1043,15 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
       parts = own;
     }
     const int BN = N >= 128 ? 128 : (N > 32 ? 64 : (N > 16 ? 32 : 16));
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
     CUtensorMap tx, tw;
     if (!make_tmap_bf16(&tx, x, d, T, kGemmBM) || !make_tmap_bf16(&tw, parts, d, 3LL * N, BN))
       return fail(BFMOE_ECUDA, "router_topk: tensor map encoding failed");
     switch (BN) {
-      case 16: e = launch_router_tc<16, 4>(tx, tw, bias, T, d, N, k, eps_c, logits, unsure, idx, gates, cc, s); break;
-      case 32: e = launch_router_tc<32, 4>(tx, tw, bias, T, d, N, k, eps_c, logits, unsure, idx, gates, cc, s); break;
-      case 64: e = launch_router_tc<64, 4>(tx, tw, bias, T, d, N, k, eps_c, logits, unsure, idx, gates, cc, s); break;
-      default: e = launch_router_tc<128, 3>(tx, tw, bias, T, d, N, k, eps_c, logits, unsure, idx, gates, cc, s); break;
+      case 16: e = launch_router_tc<16, 4>(tx, tw, bias, T, d, N, k, eps_c, logits, xb, w_gate, idx, gates, cc, s); break;
+      case 32: e = launch_router_tc<32, 4>(tx, tw, bias, T, d, N, k, eps_c, logits, xb, w_gate, idx, gates, cc, s); break;
+      case 64: e = launch_router_tc<64, 4>(tx, tw, bias, T, d, N, k, eps_c, logits, xb, w_gate, idx, gates, cc, s); break;
+      default: e = launch_router_tc<128, 3>(tx, tw, bias, T, d, N, k, eps_c, logits, xb, w_gate, idx, gates, cc, s); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "router_topk: tensor-core router");
   } else {
@@ -1077,10 +1077,11 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
     if (e != cudaSuccess) return cuda_fail(e, "router_topk: top-k");
   }
   // the tokens left undecided by the float32 top-k, settled from exact
-  // logits (usually a few per thousand; near ties always)
-  {
+  // logits (usually a few per thousand; near ties always); the tensor-core
+  // router settles its own in its epilogue
+  if (!tc_router) {
     const int g = grid_for(T, kFixWarps, sm_count());
-    int32_t* ccp = tc_router ? cc : nullptr;
+    int32_t* ccp = nullptr;
     e = launch("router_fixup", s, [&] {
       if (x_dtype == BFMOE_BF16)
         pdl_launch(router_fixup_kernel<__nv_bfloat16>, g, kFixWarps * 32, 0, s, static_cast<const __nv_bfloat16*>(x),

@@ -324,6 +324,96 @@ __global__ __launch_bounds__(256) void router_topk_kernel(const float* __restric
 constexpr int kFixWindow = 64;
 constexpr int kFixWarps = 8;
 
+// Settle token t from exact logits (steps 1-3 above), one warp: lr is its
+// row of float32 logits, idx[t][k-1] its provisional k-th pick, win a
+// per-warp buffer of kFixWindow ints.  Lane 0 writes idx and gates and, when
+// cc is given, moves the token's rows in that bucket-chunk histogram from
+// the provisional experts to the final ones.
+template <typename Tx>
+__device__ void settle_token(int t, const Tx* __restrict__ xr, const float* __restrict__ wg,
+                             const float* __restrict__ bias, const float* lr, int d, int N, int k, float eps_c,
+                             int* win, int lane, int32_t* idx, float* gates, int32_t* cc) {
+  // 1. the float32 k-th logit V: the router's provisional k-th pick is the
+  // float32 top-k's last entry; then the window
+  const int ik = idx[static_cast<size_t>(t) * k + (k - 1)];
+  float vk = ik >= 0 && ik < N ? lr[ik] : -INFINITY;
+  if (isnan(vk)) vk = -INFINITY;
+  const float thr = vk > -INFINITY ? vk - 4.f * eps_c * (1.f + fabsf(vk)) : -INFINITY;
+  int nwin = 0;
+#pragma unroll 4
+  for (int e0 = 0; e0 < N; e0 += 32) {
+    const int e = e0 + lane;
+    float l = e < N ? lr[e] : -INFINITY;
+    if (isnan(l)) l = -INFINITY;
+    const bool in = e < N && l >= thr;
+    const unsigned m = __ballot_sync(FULL_MASK, in);
+    const int pos = nwin + __popc(m & ((1u << lane) - 1u));
+    if (in && pos < kFixWindow) win[pos] = e;
+    nwin += __popc(m);
+  }
+  __syncwarp();
+  // 2. exact logits of the window (all experts when it overflows) and
+  // 3. the exact top-k
+  const bool all = nwin > kFixWindow;
+  const int cnt = all ? N : nwin;
+  float vh[BFMOE_MAX_K], vl[BFMOE_MAX_K];
+  int id[BFMOE_MAX_K];
+#pragma unroll
+  for (int j = 0; j < BFMOE_MAX_K; ++j) {
+    vh[j] = -INFINITY;
+    vl[j] = 0.f;
+    id[j] = 0x7fffffff;
+  }
+  for (int q0 = 0; q0 < cnt; q0 += 4) {
+    int es[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) es[j] = q0 + j < cnt ? (all ? q0 + j : win[q0 + j]) : -1;
+    float h4[4], l4[4];
+    df_logits4(xr, wg, bias, d, es, lane, h4, l4);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (es[j] < 0) break;
+      // every lane holds the same value: a uniform insertion
+      float ch = h4[j], cl = l4[j];
+      int ci = es[j];
+#pragma unroll
+      for (int r = 0; r < BFMOE_MAX_K; ++r) {
+        if (r < k && df_ranks_before(ch, cl, ci, vh[r], vl[r], id[r])) {
+          const float th = vh[r], tl = vl[r];
+          const int ti = id[r];
+          vh[r] = ch;
+          vl[r] = cl;
+          id[r] = ci;
+          ch = th;
+          cl = tl;
+          ci = ti;
+        }
+      }
+    }
+  }
+  if (lane == 0) {
+    // gates from the exact differences l_j - l_0
+    float z[BFMOE_MAX_K];
+    float sum = 0.f;
+    const bool finite_top = vh[0] > -INFINITY;
+    for (int j = 0; j < k; ++j) {
+      z[j] = finite_top ? expf(__fadd_rn(__fsub_rn(vh[j], vh[0]), __fsub_rn(vl[j], vl[0]))) : 1.f;
+      sum += z[j];
+    }
+    for (int j = 0; j < k; ++j) {
+      const size_t o = static_cast<size_t>(t) * k + j;
+      if (cc) {
+        const int old = idx[o];
+        if (old >= 0 && old < N) atomicSub(cc + old, 1);
+        if (id[j] >= 0 && id[j] < N) atomicAdd(cc + id[j], 1);
+      }
+      idx[o] = id[j];
+      gates[o] = z[j] / sum;
+    }
+  }
+  __syncwarp();
+}
+
 template <typename Tx>
 __global__ __launch_bounds__(kFixWarps * 32) void router_fixup_kernel(
     const Tx* __restrict__ x, const float* __restrict__ wg, const float* __restrict__ bias,
@@ -341,88 +431,8 @@ __global__ __launch_bounds__(kFixWarps * 32) void router_fixup_kernel(
       if (lane == 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(u));
       continue;
     }
-    const float* lr = logits + static_cast<size_t>(t) * N;
-    const Tx* xr = x + static_cast<size_t>(t) * d;
-    // 1. the float32 k-th logit V: the router's provisional k-th pick is
-    // the float32 top-k's last entry; then the window
-    const int ik = idx[static_cast<size_t>(t) * k + (k - 1)];
-    float vk = ik >= 0 && ik < N ? lr[ik] : -INFINITY;
-    if (isnan(vk)) vk = -INFINITY;
-    const float thr = vk > -INFINITY ? vk - 4.f * eps_c * (1.f + fabsf(vk)) : -INFINITY;
-    int nwin = 0;
-#pragma unroll 4
-    for (int e0 = 0; e0 < N; e0 += 32) {
-      const int e = e0 + lane;
-      float l = e < N ? lr[e] : -INFINITY;
-      if (isnan(l)) l = -INFINITY;
-      const bool in = e < N && l >= thr;
-      const unsigned m = __ballot_sync(FULL_MASK, in);
-      const int pos = nwin + __popc(m & ((1u << lane) - 1u));
-      if (in && pos < kFixWindow) win_s[w][pos] = e;
-      nwin += __popc(m);
-    }
-    __syncwarp();
-    // 2. exact logits of the window (all experts when it overflows) and
-    // 3. the exact top-k
-    const bool all = nwin > kFixWindow;
-    const int cnt = all ? N : nwin;
-    float vh[BFMOE_MAX_K], vl[BFMOE_MAX_K];
-    int id[BFMOE_MAX_K];
-#pragma unroll
-    for (int j = 0; j < BFMOE_MAX_K; ++j) {
-      vh[j] = -INFINITY;
-      vl[j] = 0.f;
-      id[j] = 0x7fffffff;
-    }
-    for (int q0 = 0; q0 < cnt; q0 += 4) {
-      int es[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) es[j] = q0 + j < cnt ? (all ? q0 + j : win_s[w][q0 + j]) : -1;
-      float h4[4], l4[4];
-      df_logits4(xr, wg, bias, d, es, lane, h4, l4);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (es[j] < 0) break;
-        // every lane holds the same value: a uniform insertion
-        float ch = h4[j], cl = l4[j];
-        int ci = es[j];
-#pragma unroll
-        for (int r = 0; r < BFMOE_MAX_K; ++r) {
-          if (r < k && df_ranks_before(ch, cl, ci, vh[r], vl[r], id[r])) {
-            const float th = vh[r], tl = vl[r];
-            const int ti = id[r];
-            vh[r] = ch;
-            vl[r] = cl;
-            id[r] = ci;
-            ch = th;
-            cl = tl;
-            ci = ti;
-          }
-        }
-      }
-    }
-    if (lane == 0) {
-      // gates from the exact differences l_j - l_0
-      float z[BFMOE_MAX_K];
-      float sum = 0.f;
-      const bool finite_top = vh[0] > -INFINITY;
-      for (int j = 0; j < k; ++j) {
-        z[j] = finite_top ? expf(__fadd_rn(__fsub_rn(vh[j], vh[0]), __fsub_rn(vl[j], vl[0]))) : 1.f;
-        sum += z[j];
-      }
-      for (int j = 0; j < k; ++j) {
-        const size_t o = static_cast<size_t>(t) * k + j;
-        if (chunk_counts) {
-          const int old = idx[o];
-          int32_t* cc = chunk_counts + static_cast<size_t>(t / 128) * N;
-          if (old >= 0 && old < N) atomicSub(cc + old, 1);
-          if (id[j] >= 0 && id[j] < N) atomicAdd(cc + id[j], 1);
-        }
-        idx[o] = id[j];
-        gates[o] = z[j] / sum;
-      }
-    }
-    __syncwarp();
+    settle_token(t, x + static_cast<size_t>(t) * d, wg, bias, logits + static_cast<size_t>(t) * N, d, N, k, eps_c,
+                 win_s[w], lane, idx, gates, chunk_counts ? chunk_counts + static_cast<size_t>(t / 128) * N : nullptr);
   }
 }
 

@@ -54,7 +54,8 @@ struct RouterTcCfg {
   static constexpr uint32_t BAR_BYTES = (2 * STAGES + 4) * 8 + 8;
   static constexpr uint32_t BIAS_BYTES = BFMOE_MAX_EXPERTS * 4;             // bias staged once
   static constexpr uint32_t MERGE_BYTES = kGemmBM * BFMOE_MAX_K * 8 + kGemmBM * 4;  // top-k lists, rejected maxima
-  static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + BIAS_BYTES + MERGE_BYTES;
+  static constexpr uint32_t WIN_BYTES = 4 * kFixWindow * 4;  // the settling warps' expert windows
+  static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + BIAS_BYTES + MERGE_BYTES + WIN_BYTES;
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : 256));
 };
 
@@ -106,7 +107,8 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
                                                            const __grid_constant__ CUtensorMap tmW,
                                                            const float* __restrict__ bias, int T, int d, int N,
                                                            float eps_c, float* __restrict__ logits,
-                                                           int* __restrict__ unsure_list,
+                                                           const __nv_bfloat16* __restrict__ x,
+                                                           const float* __restrict__ w_gate,
                                                            int32_t* __restrict__ idx,
                                                            float* __restrict__ gates,
                                                            int32_t* __restrict__ chunk_counts) {
@@ -122,6 +124,7 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
   float* merge_v = bias_s + BFMOE_MAX_EXPERTS;                       // [128][K]
   int* merge_i = reinterpret_cast<int*>(merge_v + kGemmBM * BFMOE_MAX_K);  // [128][K]
   float* merge_r = reinterpret_cast<float*>(merge_i + kGemmBM * BFMOE_MAX_K);  // [128]
+  int* win_s = reinterpret_cast<int*>(merge_r + kGemmBM);                      // [4][kFixWindow]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kGemmBM;
@@ -285,6 +288,7 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
   const int et = threadIdx.x - 64;  // 0 .. 255
   for (int e = et; e < N; e += kRouterEpiWarps * 32) hist[e] = 0;
   asm volatile("bar.sync 1, %0;" ::"r"(kRouterEpiWarps * 32) : "memory");
+  bool unsure = false;
   if (hf == 0 && ok && row < T) {
 #pragma unroll
     for (int j = 0; j < K; ++j) top.push(merge_v[lr * BFMOE_MAX_K + j], merge_i[lr * BFMOE_MAX_K + j]);
@@ -297,7 +301,21 @@ __global__ __launch_bounds__(kRouterThreads, 1) void router_tc_kernel(const __gr
       gates[static_cast<size_t>(row) * K + j] = g[j];
       if (top.id[j] < N) atomicAdd(&hist[top.id[j]], 1);
     }
-    if (!topk_is_clear(top.v, K, top.rej, eps_c)) unsure_list[2 + atomicAdd(unsure_list, 1)] = row;
+    unsure = !topk_is_clear(top.v, K, top.rej, eps_c);
+  }
+  if (hf == 0) {
+    // rows whose float32 top-k is undecided (a few per thousand) are settled
+    // here from exact logits, the warp working on one row at a time; the
+    // row's float32 logits were stored above and are visible to the warp
+    __syncwarp();
+    unsigned um = __ballot_sync(FULL_MASK, unsure);
+    while (um) {
+      const int src = __ffs(um) - 1;
+      um &= um - 1;
+      const int t = m0 + sp * 32 + src;
+      settle_token(t, x + static_cast<size_t>(t) * d, w_gate, bias, logits + static_cast<size_t>(t) * N, d, N, K,
+                   eps_c, win_s + sp * kFixWindow, lane, idx, gates, hist);
+    }
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kRouterEpiWarps * 32) : "memory");
   for (int e = et; e < N; e += kRouterEpiWarps * 32)
