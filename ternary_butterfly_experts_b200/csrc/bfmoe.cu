@@ -552,7 +552,7 @@ template <int D>
 cudaError_t launch_fused(const CUtensorMap& tb, const __nv_bfloat16* x, const int32_t* idx, const float* gates,
                          const int32_t* rows, const int32_t* offsets, int32_t* pad, const float4* tq,
                          const float4* pq, long long R, int k, int N, float alpha, __nv_bfloat16* slot,
-                         cudaStream_t s) {
+                         bool pad_ready, cudaStream_t s) {
   using C = FusedCfg<D>;
   static std::atomic<uint64_t> done{0};
   if (needs_attr(done)) {
@@ -566,12 +566,15 @@ cudaError_t launch_fused(const CUtensorMap& tb, const __nv_bfloat16* x, const in
   int32_t* pad_off = pad;
   int32_t* pmap = pad + (N + 1);
   int32_t* qex = pmap + cap;
-  cudaError_t e = launch("bucket_pad", s, [&] {
-    const int g = grid_for(cap, 256, sm_count() * 8);
-    pdl_launch(bucket_pad_kernel, g, 256, static_cast<size_t>(N + 1) * 8, s, offsets, rows, idx, R, N, cap, pad_off,
-               pmap, qex);
-  });
-  if (e != cudaSuccess) return e;
+  // (already written by the router's scatter when pad_ready)
+  if (!pad_ready) {
+    const cudaError_t e = launch("bucket_pad", s, [&] {
+      const int g = grid_for(cap, 256, sm_count() * 8);
+      pdl_launch(bucket_pad_kernel, g, 256, static_cast<size_t>(N + 1) * 8, s, offsets, rows, idx, R, N, cap,
+                 pad_off, pmap, qex);
+    });
+    if (e != cudaSuccess) return e;
+  }
   const int grid = static_cast<int>(std::min<long long>(cap / kGemmBM, sm_count()));
   return launch("fused_expert", s, [&] {
     pdl_launch(fused_expert_kernel<D>, grid, kFusedThreads, C::SMEM_BYTES, s, tb, x, gates,
@@ -601,7 +604,7 @@ cudaError_t launch_combine(bool bf16, bool fast, const void* slot, int T, int k,
 // holds the weight tables (TabPlan), built per call or prepared once.
 int forward_body(const bfmoe_layer* layer, const void* x, bool bf16, int T, int k, const int32_t* idx,
                  const float* gates, const int32_t* offsets, const int32_t* rows, void* y, const Plan& p, uint8_t* W,
-                 const uint8_t* tabs, cudaStream_t s) {
+                 const uint8_t* tabs, cudaStream_t s, bool pad_ready) {
   const int d = layer->d, N = layer->n_experts, L = ilog2(d);
   const TabPlan tp = make_tab_plan(d, N);
   const float2* tab_t = reinterpret_cast<const float2*>(tabs + tp.theta);
@@ -622,10 +625,10 @@ int forward_body(const bfmoe_layer* layer, const void* x, bool bf16, int T, int 
     auto* sb = static_cast<__nv_bfloat16*>(slot);
     int32_t* pad = reinterpret_cast<int32_t*>(W + p.pad);
     switch (d) {
-      case 64: e = launch_fused<64>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, s); break;
-      case 128: e = launch_fused<128>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, s); break;
-      case 256: e = launch_fused<256>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, s); break;
-      default: e = launch_fused<512>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, s); break;
+      case 64: e = launch_fused<64>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, pad_ready, s); break;
+      case 128: e = launch_fused<128>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, pad_ready, s); break;
+      case 256: e = launch_fused<256>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, pad_ready, s); break;
+      default: e = launch_fused<512>(tb, xb, idx, gates, rows, offsets, pad, tq, pq, R, k, N, layer->alpha, sb, pad_ready, s); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "forward: fused expert kernel");
     e = launch_combine(true, true, slot, T, k, d, y, s);
@@ -988,7 +991,7 @@ cudaError_t split_gate_weights(const float* w_gate, int N, int d, __nv_bfloat16*
 // same weights does once.
 int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_gate, const float* bias, int n_experts,
                      int k, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, int32_t* rows, void* ws,
-                     size_t ws_bytes, cudaStream_t s, const __nv_bfloat16* parts_ready);
+                     size_t ws_bytes, cudaStream_t s, const __nv_bfloat16* parts_ready, int32_t* pad_out = nullptr);
 
 }  // namespace
 
@@ -1003,7 +1006,7 @@ namespace {
 
 int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_gate, const float* bias, int n_experts,
                      int k, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, int32_t* rows, void* ws,
-                     size_t ws_bytes, cudaStream_t s, const __nv_bfloat16* parts_ready) {
+                     size_t ws_bytes, cudaStream_t s, const __nv_bfloat16* parts_ready, int32_t* pad_out) {
   int rc = check_sizes(d, n_experts, T, k);
   if (rc) return rc;
   if ((rc = check_dtype(x_dtype))) return rc;
@@ -1102,7 +1105,7 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
   if (needs_attr(done)) {
     cudaFuncSetAttribute(bucket_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BFMOE_MAX_EXPERTS * 4);
     cudaFuncSetAttribute(bucket_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         BFMOE_MAX_EXPERTS * 36 + 16);
+                         BFMOE_MAX_EXPERTS * 40 + 32);
     attr_set(done);
   }
   if (!tc_router) {  // the tensor-core router writes the chunk histograms itself
@@ -1111,9 +1114,10 @@ int router_topk_impl(const void* x, int x_dtype, int T, int d, const float* w_ga
   }
   e = launch("bucket_scan", s, [&] { pdl_launch(bucket_scan_kernel, (N + 31) / 32, 1024, 0, s, cc, nchunks, N, totals); });
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scan");
-  const size_t scatter_smem = ((N + 1) * 4 + 15) / 16 * 16 + static_cast<size_t>(N) * 32;
+  const size_t scatter_smem = ((N + 1) * 4 + 15) / 16 * 16 + static_cast<size_t>(N) * 36 + 4;
   e = launch("bucket_scatter", s, [&] {
-    pdl_launch(bucket_scatter_kernel, nchunks, chunk, scatter_smem, s, idx, R, N, cc, totals, counts, offsets, rows);
+    pdl_launch(bucket_scatter_kernel, nchunks, chunk, scatter_smem, s, idx, R, N, static_cast<const int32_t*>(cc),
+               static_cast<const int32_t*>(totals), counts, offsets, rows, pad_out, pad_cap(R, N));
   });
   if (e != cudaSuccess) return cuda_fail(e, "router_topk: bucket scatter");
   return ok();
@@ -1186,7 +1190,7 @@ int bfmoe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int T, i
     if ((rc = build_weight_tables(layer, W + p.tabs, s))) return rc;
     tabs = W + p.tabs;
   }
-  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, tabs, s);
+  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, tabs, s, false);
 }
 
 size_t bfmoe_moe_host_workspace_size(int d, int n_experts, int T, int k, int x_dtype, int chunk) {
@@ -1258,12 +1262,15 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
       rc = cuda_fail(e, "moe_forward_host: copy in");
       break;
     }
+    // the router's scatter also writes the fused kernel's padded bucket order
+    const Plan pcur = make_plan(d, N, Tc, k, x_dtype);
+    const bool fused = fused_path(x_dtype, d);
     rc = router_topk_impl(x_dev + o, x_dtype, Tc, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows,
-                          Wm + pc.fwd_end, pc.rt_end, s, parts);
+                          Wm + pc.fwd_end, pc.rt_end, s, parts,
+                          fused ? reinterpret_cast<int32_t*>(Wm + pcur.pad) : nullptr);
     if (c == 0 && (e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) rc = cuda_fail(e, "moe_forward_host: join");
     if (rc) break;
-    rc = forward_body(layer, x_dev + o, bf16, Tc, k, idx, gates, offsets, rows, y_dev + o,
-                      make_plan(d, N, Tc, k, x_dtype), Wm, tabs, s);
+    rc = forward_body(layer, x_dev + o, bf16, Tc, k, idx, gates, offsets, rows, y_dev + o, pcur, Wm, tabs, s, fused);
     if (rc) break;
     if ((e = cudaEventRecord(pipe->ev_out[c], s)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(pipe->out, pipe->ev_out[c], 0)) != cudaSuccess ||
@@ -1302,12 +1309,15 @@ int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int 
     return bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, nullptr, 0,
                              stream);
   const uint8_t* tabs = static_cast<const uint8_t*>(layer->tables);
+  // the router's scatter also writes the fused kernel's padded bucket order
+  const bool fused = fused_path(x_dtype, d);
+  int32_t* pad = fused ? reinterpret_cast<int32_t*>(W + p.pad) : nullptr;
   if (tabs) {
     // prepared tables: router and forward in stream order, nothing on the side
-    rc = bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, W + p.fwd_end,
-                           p.rt_end, stream);
+    rc = router_topk_impl(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, W + p.fwd_end,
+                          p.rt_end, s, nullptr, pad);
     if (rc) return rc;
-    return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, tabs, s);
+    return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, tabs, s, fused);
   }
   // fork: the weight-derived tables build on the side stream while the router runs
   SideStream* ss = nullptr;
@@ -1317,12 +1327,12 @@ int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int 
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward: fork");
   if ((rc = build_weight_tables(layer, W + p.tabs, ss->stream))) return rc;
   if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return cuda_fail(e, "moe_forward: join record");
-  rc = bfmoe_router_topk(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, W + p.fwd_end,
-                         p.rt_end, stream);
+  rc = router_topk_impl(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, W + p.fwd_end,
+                        p.rt_end, s, nullptr, pad);
   // join before anything else can fail, so the side stream never outlives the call's work
   if ((e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) return cuda_fail(e, "moe_forward: join");
   if (rc) return rc;
-  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, W + p.tabs, s);
+  return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, W + p.tabs, s, fused);
 }
 
 size_t bfmoe_layer_tables_size(int d, int n_experts) {

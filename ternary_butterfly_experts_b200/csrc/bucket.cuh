@@ -119,25 +119,51 @@ __device__ __forceinline__ void block_exclusive_scan(F val, int N, int* off) {
 
 // Every block scans the per-expert totals itself (N <= 4096 ints), so the
 // offsets need no launch of their own; block 0 also writes counts and
-// offsets out.
+// offsets out; block b reads its chunk's prefixes from chunk_prefix
+// (bucket_scan_kernel).  With pad given ([N+1] padded offsets, then [p_cap]
+// row map, then [p_cap / 32] quadrant experts), the blocks also write the
+// padded bucket order that bucket_pad_kernel would build from the buckets.
 __global__ __launch_bounds__(1024) void bucket_scatter_kernel(const int32_t* __restrict__ idx, long long R, int N,
                                                               const int32_t* __restrict__ chunk_prefix,
                                                               const int32_t* __restrict__ totals,
                                                               int32_t* __restrict__ counts_out,
                                                               int32_t* __restrict__ offsets_out,
-                                                              int32_t* __restrict__ rows) {
+                                                              int32_t* __restrict__ rows, int32_t* __restrict__ pad,
+                                                              long long p_cap) {
   extern __shared__ uint8_t scatter_smem[];
   int* off = reinterpret_cast<int*>(scatter_smem);                   // [N+1]
   uint8_t* wcnt = scatter_smem + ((N + 1) * 4 + 15) / 16 * 16;       // [N][32]: rows of expert e in warp w
+  int* poff = reinterpret_cast<int*>(wcnt + static_cast<size_t>(N) * 32);  // [N+1] (padded order only)
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   for (int q = tid; q < N * 8; q += blockDim.x) reinterpret_cast<uint32_t*>(wcnt)[q] = 0u;
   pdl_wait();
   pdl_trigger();
   block_exclusive_scan([&](int e) { return totals[e]; }, N, off);
+  int32_t* pmap = nullptr;
+  if (pad) {
+    // the padded order: every bucket rounded up to 32 rows; this block fills
+    // the padding and quadrant experts of experts b, b + gridDim.x, ... and
+    // its share of the tail up to p_cap
+    block_exclusive_scan([&](int e) { return (off[e + 1] - off[e] + 31) & ~31; }, N, poff);
+    pmap = pad + (N + 1);
+    int32_t* qex = pmap + p_cap;
+    if (blockIdx.x == 0)
+      for (int e = tid; e <= N; e += blockDim.x) pad[e] = poff[e];
+    for (int e = blockIdx.x; e < N; e += gridDim.x) {
+      const int p0 = poff[e], c = off[e + 1] - off[e], p1 = poff[e + 1];
+      for (int q = tid; q < p1 - p0 - c; q += blockDim.x) pmap[p0 + c + q] = -1;
+      for (int q = tid; q < (p1 - p0) / 32; q += blockDim.x) qex[p0 / 32 + q] = e;
+    }
+    for (long long P = poff[N] + static_cast<long long>(blockIdx.x) * blockDim.x + tid; P < p_cap;
+         P += static_cast<long long>(gridDim.x) * blockDim.x) {
+      pmap[P] = -1;
+      if ((P & 31) == 0) qex[P >> 5] = -1;
+    }
+  }
   if (blockIdx.x == 0) {
     for (int e = tid; e <= N; e += blockDim.x) {
       offsets_out[e] = off[e];
-      if (e < N) counts_out[e] = totals[e];
+      if (e < N) counts_out[e] = off[e + 1] - off[e];
     }
   }
   const long long r = static_cast<long long>(blockIdx.x) * blockDim.x + tid;
@@ -162,6 +188,7 @@ __global__ __launch_bounds__(1024) void bucket_scatter_kernel(const int32_t* __r
   if (valid) {
     const int pos = off[e] + chunk_prefix[static_cast<size_t>(blockIdx.x) * N + e] + before + rank;
     rows[pos] = static_cast<int32_t>(r);
+    if (pmap) pmap[poff[e] + (pos - off[e])] = static_cast<int32_t>(r);
   }
 }
 

@@ -239,8 +239,12 @@ def test_bad_routing_is_reported_not_faulted():
 
 # -- the combined call -------------------------------------------------------------
 
-@pytest.mark.parametrize("d,N,k,T,dt", [(512, 64, 2, 777, "bf16"), (64, 8, 2, 256, "f32"), (32, 4, 3, 50, "bf16")])
+@pytest.mark.parametrize("d,N,k,T,dt", [(512, 64, 2, 777, "bf16"), (64, 8, 2, 256, "f32"), (32, 4, 3, 50, "bf16"),
+                                         # many experts, and many chunks
+                                         (256, 256, 2, 2000, "bf16"), (128, 256, 2, 40000, "bf16")])
 def test_moe_forward_equals_router_then_forward(d, N, k, T, dt):
+    """The combined call (whose router scatter also writes the fused kernel's
+    padded bucket order) equals the router then the forward bit for bit."""
     m = B()
     wl = W.custom("mf", d=d, n_experts=N, k=k, tokens=T, dtype=dt, bias_var=0.5)
     inp = W.generate(wl, seed=d + T)
