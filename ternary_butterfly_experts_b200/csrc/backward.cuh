@@ -18,10 +18,12 @@
 //     p = c p' + sg s q',   q = -sg s p' + c q'   (the same for the gradients).
 //
 // Layout: one warp per routed row; lane l holds the E = max(1, d/32)
-// consecutive elements [l E, l E + E) of the row's value and gradient.  One
-// CTA per expert walks that expert's bucket; the angle gradients of a stage
-// are summed in shared memory ([L][d/2] float32) with shared atomics (their
-// order, and so the last bits, varies between runs) and written once.
+// consecutive elements [l E, l E + E) of the row's value and gradient.
+// gridDim.y CTAs per expert share that expert's bucket (warp w of CTA y takes
+// the rows y*8 + w, y*8 + w + 8*gridDim.y, ...); a CTA sums the angle
+// gradients of its rows in shared memory ([L][d/2] float32, shared atomics)
+// and adds them to the expert's (zeroed) gradient with global atomics.  The
+// order of the additions, and so the last bits, varies between runs.
 #pragma once
 #include "common.cuh"
 #include "rotate.cuh"
@@ -167,10 +169,10 @@ __device__ __forceinline__ void bw_store(float* __restrict__ dst, const float (&
   for (int q = 0; q < E; ++q) dst[lane * E + q] = v[q];
 }
 
-// Output side, one CTA per expert e: for its rows (bucket position p, row
+// Output side, gridDim.y CTAs per expert e: for its rows (bucket position p, row
 // r = rows[p], token t = r / k), from z = Z[p]: v = B(phi) z, dg[r] = <v, gy_t>,
 // dv = gates[r] gy_t, then back through B(phi): dZ[p] = B(phi)^T dv and
-// dphi[e] (written whole: zero for an expert without rows).
+// dphi[e] (added to the zeroed gradient).
 template <int E>
 __global__ __launch_bounds__(256) void bw_post_kernel(const float* __restrict__ Z, const float* __restrict__ gy,
                                                       const int32_t* __restrict__ rows,
@@ -191,7 +193,7 @@ __global__ __launch_bounds__(256) void bw_post_kernel(const float* __restrict__ 
   if (p0 < 0 || p1 < p0 || p1 > R) {
     if (threadIdx.x == 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(e));
   } else {
-    for (int p = p0 + w; p < p1; p += nw) {
+    for (int p = p0 + blockIdx.y * nw + w; p < p1; p += nw * gridDim.y) {
       const int r = rows[p];
       if (r < 0 || r >= R) {
         if (lane == 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
@@ -217,10 +219,11 @@ __global__ __launch_bounds__(256) void bw_post_kernel(const float* __restrict__ 
   }
   __syncthreads();
   float* out = dphi + static_cast<size_t>(e) * L * half;
-  for (int i = threadIdx.x; i < L * half; i += blockDim.x) out[i] = acc[i];
+  for (int i = threadIdx.x; i < L * half; i += blockDim.x)
+    if (acc[i] != 0.f) atomicAdd(out + i, acc[i]);
 }
 
-// Input side, one CTA per expert e: for its rows, from u = U[p] and
+// Input side, gridDim.y CTAs per expert e: for its rows, from u = U[p] and
 // du = dU[p], back through B(theta)^T (stages 0 .. L-1, blocks transposed):
 // dXr[r] = B(theta) du and dtheta[e].
 template <int E>
@@ -241,7 +244,7 @@ __global__ __launch_bounds__(256) void bw_pre_kernel(const float* __restrict__ U
   if (p0 < 0 || p1 < p0 || p1 > R) {
     if (threadIdx.x == 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(e));
   } else {
-    for (int p = p0 + w; p < p1; p += nw) {
+    for (int p = p0 + blockIdx.y * nw + w; p < p1; p += nw * gridDim.y) {
       const int r = rows[p];
       if (r < 0 || r >= R) {
         if (lane == 0) report_error(BFMOE_EDEVICE_BOUNDS, static_cast<unsigned>(p));
@@ -256,7 +259,8 @@ __global__ __launch_bounds__(256) void bw_pre_kernel(const float* __restrict__ U
   }
   __syncthreads();
   float* out = dtheta + static_cast<size_t>(e) * L * half;
-  for (int i = threadIdx.x; i < L * half; i += blockDim.x) out[i] = acc[i];
+  for (int i = threadIdx.x; i < L * half; i += blockDim.x)
+    if (acc[i] != 0.f) atomicAdd(out + i, acc[i]);
 }
 
 // 2-bit codes of W^T: wt[i][o] = w[o][i] (the base read by columns, for
@@ -394,35 +398,57 @@ __global__ __launch_bounds__(256) void bw_token_kernel(const float* __restrict__
 }
 
 // Router weights, one CTA per expert: dW_g[e] = sum over the expert's bucket
-// (ascending tokens) of dl_r x_t, db[e] = sum of dl_r.
+// (ascending tokens) of dl_r x_t, db[e] = sum of dl_r.  The bucket's tokens
+// and dl are staged in shared memory 256 rows at a time; thread c sums the
+// columns c, c + 256, ... in bucket order (the x loads of successive rows
+// are independent, so many are in flight).
+constexpr int kRouterGradCols = BFMOE_MAX_D / 256;
 template <typename Tx>
 __global__ __launch_bounds__(256) void bw_router_kernel(const Tx* __restrict__ x, const float* __restrict__ dl,
                                                         const int32_t* __restrict__ rows,
                                                         const int32_t* __restrict__ offsets, int k, int d,
                                                         long long R, float* __restrict__ dw_gate,
                                                         float* __restrict__ dbias) {
+  __shared__ int s_tok[256];
+  __shared__ float s_dl[256];
   const int e = blockIdx.x;
   const int p0 = offsets[e], p1 = offsets[e + 1];
   const bool ok = p0 >= 0 && p1 >= p0 && p1 <= R;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float s = 0.f;
-    if (ok)
-      for (int p = p0; p < p1; ++p) {
-        const int r = rows[p];
-        if (r < 0 || r >= R) continue;
-        s += dl[r] * to_f32(x[static_cast<size_t>(r / k) * d + c]);
+  float acc[kRouterGradCols];
+#pragma unroll
+  for (int m = 0; m < kRouterGradCols; ++m) acc[m] = 0.f;
+  float db = 0.f;
+  for (int base = ok ? p0 : p1; base < p1; base += 256) {
+    const int n = p1 - base < 256 ? p1 - base : 256;
+    if (static_cast<int>(threadIdx.x) < n) {
+      const int r = rows[base + threadIdx.x];
+      const bool valid = r >= 0 && r < R;
+      s_tok[threadIdx.x] = valid ? r / k : -1;
+      s_dl[threadIdx.x] = valid ? dl[r] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int j = 0; j < n; ++j) {
+      const int t = s_tok[j];
+      if (t < 0) continue;
+      const float g = s_dl[j];
+      const Tx* xr = x + static_cast<size_t>(t) * d;
+#pragma unroll
+      for (int m = 0; m < kRouterGradCols; ++m) {
+        const int c = threadIdx.x + 256 * m;
+        if (c < d) acc[m] += g * to_f32(xr[c]);
       }
-    dw_gate[static_cast<size_t>(e) * d + c] = s;
+    }
+    if (threadIdx.x == 0)
+      for (int j = 0; j < n; ++j) db += s_dl[j];
+    __syncthreads();
   }
-  if (dbias && threadIdx.x == 0) {
-    float s = 0.f;
-    if (ok)
-      for (int p = p0; p < p1; ++p) {
-        const int r = rows[p];
-        if (r >= 0 && r < R) s += dl[r];
-      }
-    dbias[e] = s;
+#pragma unroll
+  for (int m = 0; m < kRouterGradCols; ++m) {
+    const int c = threadIdx.x + 256 * m;
+    if (c < d) dw_gate[static_cast<size_t>(e) * d + c] = acc[m];
   }
+  if (dbias && threadIdx.x == 0) dbias[e] = db;
 }
 
 }  // namespace bfmoe

@@ -889,12 +889,21 @@ struct BwRows {
                                                                   k, d, L, N, U);
       });
     }
-    if (stage == 1)
+    // CTAs per expert: about 16 rows each on average (2 per warp)
+    const long long per_expert = (R + N - 1) / N;
+    const dim3 grid(N, static_cast<unsigned>(std::min<long long>(64, std::max<long long>(1, (per_expert + 15) / 16))));
+    const size_t ang = static_cast<size_t>(N) * L * (d / 2) * sizeof(float);
+    if (stage == 1) {
+      cudaError_t e = cudaMemsetAsync(dphi, 0, ang, s);
+      if (e != cudaSuccess) return e;
       return launch("bw_post", s, [&] {
-        bw_post_kernel<E><<<N, 256, smem, s>>>(Z, gy, rows, offsets, gates, tab_p, d, L, k, N, R, Z, dg, dphi);
+        bw_post_kernel<E><<<grid, 256, smem, s>>>(Z, gy, rows, offsets, gates, tab_p, d, L, k, N, R, Z, dg, dphi);
       });
+    }
+    cudaError_t e = cudaMemsetAsync(dtheta, 0, ang, s);
+    if (e != cudaSuccess) return e;
     return launch("bw_pre", s, [&] {
-      bw_pre_kernel<E><<<N, 256, smem, s>>>(U, dU, rows, offsets, tab_t, d, L, R, Z, dtheta);
+      bw_pre_kernel<E><<<grid, 256, smem, s>>>(U, dU, rows, offsets, tab_t, d, L, R, Z, dtheta);
     });
   }
 };
