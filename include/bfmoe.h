@@ -75,6 +75,9 @@ typedef struct {
   const void* tables;         /* NULL, or this layer's weight tables written by
                                  bfmoe_prepare_layer (then the calls read them
                                  instead of rebuilding them per call)               */
+  const void* gate_parts;     /* NULL, or the router weights passed to the
+                                 bfmoe_moe_* calls split by bfmoe_prepare_gate
+                                 (then those calls skip the per-call split)         */
 } bfmoe_layer;
 
 /*
@@ -194,6 +197,26 @@ int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int 
                       const float* w_gate, const float* bias, int k,
                       int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, int32_t* rows,
                       void* y, void* ws, size_t ws_bytes, bfmoe_stream_t stream);
+
+/*
+ * Split the router weights once for the tensor-core router (no counterpart
+ * on the pages).  The bf16 router multiplies x by an exact three-part bf16
+ * split of the float32 W_g (hi + mid + lo == W_g); without prepared parts
+ * every call makes it.  With `layer->gate_parts` pointing at memory written
+ * here from the same w_gate, bfmoe_moe_forward and bfmoe_moe_forward_host
+ * use it instead (results identical bit for bit); they ignore it on the
+ * paths that do not split (float32 x, d not a multiple of 64).  Redo after
+ * changing W_g.
+ *   w_gate    device float [N][d]
+ *   parts     device memory of bfmoe_gate_parts_size(N, d) bytes, 256-byte
+ *             aligned (written: [3][N][d] bfloat16)
+ * Returns BFMOE_EINVAL / BFMOE_EWORKSPACE on bad arguments (nothing launched).
+ */
+int bfmoe_prepare_gate(const float* w_gate, int n_experts, int d, void* parts, size_t bytes,
+                       bfmoe_stream_t stream);
+
+/* Bytes that bfmoe_prepare_gate writes (0 for invalid sizes). */
+size_t bfmoe_gate_parts_size(int n_experts, int d);
 
 /*
  * Build a layer's weight tables once (no counterpart on the pages, which store

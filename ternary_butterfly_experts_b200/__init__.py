@@ -22,7 +22,7 @@ from .capi import BFMOE_BF16, BFMOE_F32, BfmoeError
 __all__ = [
     "BfmoeError", "Layer", "ButterflyMoE", "bfmoe_pack_base", "bfmoe_unpack_base", "bfmoe_router_topk",
     "bfmoe_router_topk_noalloc", "bfmoe_moe_forward", "bfmoe_moe_workspace_size", "bfmoe_prepare_layer",
-    "bfmoe_layer_tables_size", "bfmoe_backward", "bfmoe_backward_workspace_size",
+    "bfmoe_layer_tables_size", "bfmoe_prepare_gate", "bfmoe_gate_parts_size", "bfmoe_backward", "bfmoe_backward_workspace_size",
     "bfmoe_forward", "bfmoe_decode_forward", "bfmoe_materialize_expert", "bfmoe_workspace_size", "bfmoe_router_scratch_size", "bfmoe_check_device_error",
     "bfmoe_launch_count", "bfmoe_profile_enable", "bfmoe_profile_collect", "bfmoe_last_error", "workspace",
 ]
@@ -183,8 +183,9 @@ class Layer:
         self.w_packed, self.theta, self.phi = w_packed, theta, phi
         self.alpha = float(alpha)
         self.c = capi.BfmoeLayer(self.d, self.n_experts, w_packed.data_ptr(), ctypes.c_float(alpha),
-                                 theta.data_ptr(), phi.data_ptr(), None)
+                                 theta.data_ptr(), phi.data_ptr(), None, None)
         self.tables = None
+        self.gate_parts = None
 
     def prepare(self, stream=None):
         """Build the weight tables once (bfmoe_prepare_layer); later calls with
@@ -203,6 +204,25 @@ class Layer:
         self.tables = None
         return self
 
+    def prepare_gate(self, w_gate, stream=None):
+        """Split the router weights once (bfmoe_prepare_gate); the combined
+        calls with this layer and the same w_gate then skip the split."""
+        torch = _torch()
+        _need(w_gate, "w_gate", torch.float32)
+        N, d = w_gate.shape
+        n = int(capi.lib().bfmoe_gate_parts_size(N, d))
+        self.gate_parts = torch.empty(max(n, 256), dtype=torch.uint8, device=w_gate.device)
+        capi.check(capi.lib().bfmoe_prepare_gate(_ptr(w_gate), N, d, _ptr(self.gate_parts), self.gate_parts.numel(),
+                                                _stream(stream)))
+        self.c.gate_parts = self.gate_parts.data_ptr()
+        return self
+
+    def unprepare_gate(self):
+        """Go back to splitting the router weights per call."""
+        self.c.gate_parts = None
+        self.gate_parts = None
+        return self
+
     @classmethod
     def from_host(cls, w_base, alpha, theta, phi, device="cuda", stream=None):
         """Pack an int8 ternary base and upload float32 angles."""
@@ -212,6 +232,17 @@ class Layer:
         th = torch.as_tensor(theta, dtype=torch.float32).to(device).contiguous()
         ph = torch.as_tensor(phi, dtype=torch.float32).to(device).contiguous()
         return cls(packed, float(alpha), th, ph)
+
+
+def bfmoe_gate_parts_size(n_experts: int, d: int) -> int:
+    return int(capi.lib().bfmoe_gate_parts_size(n_experts, d))
+
+
+def bfmoe_prepare_gate(w_gate, parts, stream=None):
+    """Write the exact bf16 split of w_gate [N][d] into parts (device bytes)."""
+    N, d = w_gate.shape
+    capi.check(capi.lib().bfmoe_prepare_gate(_ptr(w_gate), N, d, _ptr(parts), parts.numel(), _stream(stream)))
+    return parts
 
 
 def bfmoe_layer_tables_size(d: int, n_experts: int) -> int:

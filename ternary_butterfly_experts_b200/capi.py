@@ -32,7 +32,7 @@ STATUS_NAMES = {0: "OK", 1: "EINVAL", 2: "ENOT_TERNARY", 3: "EUNSUPPORTED", 4: "
 class BfmoeLayer(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int), ("n_experts", ctypes.c_int), ("w_packed", ctypes.c_void_p),
                 ("alpha", ctypes.c_float), ("theta", ctypes.c_void_p), ("phi", ctypes.c_void_p),
-                ("tables", ctypes.c_void_p)]
+                ("tables", ctypes.c_void_p), ("gate_parts", ctypes.c_void_p)]
 
 
 class BfmoeKernelTime(ctypes.Structure):
@@ -69,6 +69,8 @@ SIGNATURES = {
     "bfmoe_moe_host_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "bfmoe_materialize_expert": (_I, [ctypes.POINTER(BfmoeLayer), _I, _P, _P]),
     "bfmoe_decode_forward": (_I, [ctypes.POINTER(BfmoeLayer), _P, _I, _I, _I, _P, _P, _P, _P]),
+    "bfmoe_prepare_gate": (_I, [_P, _I, _I, _P, _SZ, _P]),
+    "bfmoe_gate_parts_size": (_SZ, [_I, _I]),
     "bfmoe_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "bfmoe_router_scratch_size": (_SZ, [_I, _I, _I, _I, _I]),
     "bfmoe_last_error": (ctypes.c_char_p, []),

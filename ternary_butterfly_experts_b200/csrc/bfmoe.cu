@@ -1257,10 +1257,15 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
   }
   if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return cuda_fail(e, "moe_forward_host: join record");
   // W_g is split once for all chunks, while the first chunk is copied in
-  __nv_bfloat16* parts = nullptr;
+  const __nv_bfloat16* parts = nullptr;
   if (rc == BFMOE_OK && tc_router_path(x_dtype, d)) {
-    parts = reinterpret_cast<__nv_bfloat16*>(W + hp.parts);
-    if ((e = split_gate_weights(w_gate, N, d, parts, s)) != cudaSuccess) rc = cuda_fail(e, "moe_forward_host: split");
+    if (layer->gate_parts) {
+      parts = static_cast<const __nv_bfloat16*>(layer->gate_parts);
+    } else {
+      auto* own = reinterpret_cast<__nv_bfloat16*>(W + hp.parts);
+      if ((e = split_gate_weights(w_gate, N, d, own, s)) != cudaSuccess) rc = cuda_fail(e, "moe_forward_host: split");
+      parts = own;
+    }
   }
   for (int c = 0; c < hp.nchunks && rc == BFMOE_OK; ++c) {
     const int t0 = hp.start[c], Tc = hp.start[c + 1] - t0;
@@ -1321,10 +1326,11 @@ int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int 
   // the router's scatter also writes the fused kernel's padded bucket order
   const bool fused = fused_path(x_dtype, d);
   int32_t* pad = fused ? reinterpret_cast<int32_t*>(W + p.pad) : nullptr;
+  const auto* gate_parts = static_cast<const __nv_bfloat16*>(layer->gate_parts);
   if (tabs) {
     // prepared tables: router and forward in stream order, nothing on the side
     rc = router_topk_impl(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, W + p.fwd_end,
-                          p.rt_end, s, nullptr, pad);
+                          p.rt_end, s, gate_parts, pad);
     if (rc) return rc;
     return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, tabs, s, fused);
   }
@@ -1337,11 +1343,28 @@ int bfmoe_moe_forward(const bfmoe_layer* layer, const void* x, int x_dtype, int 
   if ((rc = build_weight_tables(layer, W + p.tabs, ss->stream))) return rc;
   if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return cuda_fail(e, "moe_forward: join record");
   rc = router_topk_impl(x, x_dtype, T, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows, W + p.fwd_end,
-                        p.rt_end, s, nullptr, pad);
+                        p.rt_end, s, gate_parts, pad);
   // join before anything else can fail, so the side stream never outlives the call's work
   if ((e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) return cuda_fail(e, "moe_forward: join");
   if (rc) return rc;
   return forward_body(layer, x, x_dtype == BFMOE_BF16, T, k, idx, gates, offsets, rows, y, p, W, W + p.tabs, s, fused);
+}
+
+size_t bfmoe_gate_parts_size(int n_experts, int d) {
+  if (d < 4 || d > BFMOE_MAX_D || !is_pow2(d) || n_experts < 1 || n_experts > BFMOE_MAX_EXPERTS) return 0;
+  return static_cast<size_t>(3) * n_experts * d * sizeof(__nv_bfloat16);
+}
+
+int bfmoe_prepare_gate(const float* w_gate, int n_experts, int d, void* parts, size_t bytes, bfmoe_stream_t stream) {
+  if (!w_gate || !parts) return fail(BFMOE_EINVAL, "prepare_gate: NULL pointer");
+  if (d < 4 || d > BFMOE_MAX_D || !is_pow2(d)) return fail(BFMOE_EINVAL, "prepare_gate: bad d=%d", d);
+  if (n_experts < 1 || n_experts > BFMOE_MAX_EXPERTS) return fail(BFMOE_EINVAL, "prepare_gate: n_experts=%d", n_experts);
+  if (reinterpret_cast<uintptr_t>(parts) & 255u) return fail(BFMOE_EWORKSPACE, "prepare_gate: parts must be 256-byte aligned");
+  const size_t need = bfmoe_gate_parts_size(n_experts, d);
+  if (bytes < need) return fail(BFMOE_EWORKSPACE, "prepare_gate: %zu bytes given, %zu needed", bytes, need);
+  const cudaError_t e = split_gate_weights(w_gate, n_experts, d, static_cast<__nv_bfloat16*>(parts),
+                                           reinterpret_cast<cudaStream_t>(stream));
+  return e != cudaSuccess ? cuda_fail(e, "prepare_gate") : ok();
 }
 
 size_t bfmoe_layer_tables_size(int d, int n_experts) {

@@ -316,3 +316,38 @@ def test_prepared_tables_give_identical_results(d, N, k, T, dt):
             assert np.array_equal(yy.float().cpu().numpy().astype(np.float64), gpu["y"])
     finally:
         layer.unprepare()
+
+
+@pytest.mark.parametrize("d,N,k,T", [(512, 256, 2, 3000), (1024, 64, 2, 700)])
+def test_prepared_gate_parts_give_identical_results(d, N, k, T):
+    """Router weights split once (bfmoe_prepare_gate): the combined call and
+    the host call equal the per-call split bit for bit."""
+    m = B()
+    wl = W.custom("pg", d=d, n_experts=N, k=k, tokens=T, dtype="bf16", bias_var=0.5)
+    inp = W.generate(wl, seed=d + N)
+    layer = m.Layer.from_host(inp.w_base, inp.alpha, inp.theta, inp.phi)
+    x = inp.x.cuda().contiguous()
+    wg = torch.from_numpy(inp.w_gate).cuda()
+    bias = torch.from_numpy(inp.bias).cuda()
+    ws = torch.empty(m.bfmoe_moe_workspace_size(d, N, T, k, m.BFMOE_BF16), dtype=torch.uint8, device="cuda")
+    model = m.ButterflyMoE(layer, wg, bias, k, T, torch.bfloat16)
+    x_host = inp.x.contiguous().pin_memory()
+
+    def host_call():
+        y_host = torch.empty(x.shape, dtype=torch.bfloat16).pin_memory()
+        model.forward_host(x_host, y_host)
+        torch.cuda.synchronize()
+        return y_host
+
+    y0, r0 = m.bfmoe_moe_forward(layer, x, wg, bias, k, ws)
+    y0, i0 = y0.clone(), r0[0].clone()
+    yh0 = host_call()
+    layer.prepare_gate(wg)
+    try:
+        y1, r1 = m.bfmoe_moe_forward(layer, x, wg, bias, k, ws)
+        m.bfmoe_check_device_error()
+        assert torch.equal(r1[0], i0) and torch.equal(y1, y0)
+        # the host call cuts the tokens into chunks: compared with itself
+        assert torch.equal(host_call(), yh0)
+    finally:
+        layer.unprepare_gate()
