@@ -68,6 +68,7 @@ CASES = [
     ("d64_n8_k2", 64, 8, 2, 64, "f32"),  # the float32 headline family
     ("d256_n16_k2", 256, 16, 2, 33, "bf16"),
     ("d2048_n16_k4", 2048, 16, 4, 9, "bf16"),
+    ("d4096_n8_k8", 4096, 8, 8, 3, "f32"),  # slots in two passes of four (shared-memory bound)
 ]
 
 
