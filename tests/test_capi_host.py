@@ -100,3 +100,27 @@ def test_router_rejects_partial_bucket_outputs():
     rc = L.bfmoe_router_topk(p, 1, 0, 64, p, None, 4, 2, p, p, p, None, None, p, 64, None)
     assert rc == 1  # BFMOE_EINVAL
     assert b"all given or all NULL" in L.bfmoe_last_error()
+
+
+def test_prepare_gate_sizes_and_argument_checks():
+    """bfmoe_gate_parts_size and bfmoe_prepare_gate's checks (before any launch)."""
+    import ctypes
+    L = capi.lib()
+    assert L.bfmoe_gate_parts_size(256, 512) == 3 * 256 * 512 * 2
+    assert L.bfmoe_gate_parts_size(0, 512) == 0 and L.bfmoe_gate_parts_size(4, 100) == 0
+    assert L.bfmoe_prepare_gate(None, 4, 64, 256, 1 << 20, None) == capi.BFMOE_EINVAL
+    assert L.bfmoe_prepare_gate(16, 4, 63, 256, 1 << 20, None) == capi.BFMOE_EINVAL
+    assert L.bfmoe_prepare_gate(16, 4, 64, 16, 1 << 20, None) == capi.BFMOE_EWORKSPACE   # not 256-byte aligned
+    assert L.bfmoe_prepare_gate(16, 4, 64, 256, 100, None) == capi.BFMOE_EWORKSPACE      # too small
+
+
+def test_decode_forward_argument_checks():
+    import ctypes
+    L = capi.lib()
+    lay = capi.BfmoeLayer(64, 4, 16, ctypes.c_float(0.1), 16, 16)
+    f = L.bfmoe_decode_forward
+    assert f(None, 16, 1, 4, 2, 16, 16, 16, None) == capi.BFMOE_EINVAL                 # no layer
+    assert f(ctypes.byref(lay), 16, 1, 4, 5, 16, 16, 16, None) == capi.BFMOE_EINVAL    # k > N
+    assert f(ctypes.byref(lay), 16, 7, 4, 2, 16, 16, 16, None) == capi.BFMOE_EINVAL    # bad dtype
+    assert f(ctypes.byref(lay), None, 1, 4, 2, 16, 16, 16, None) == capi.BFMOE_EINVAL  # NULL x
+    assert f(ctypes.byref(lay), None, 1, 0, 2, None, None, None, None) == capi.BFMOE_OK  # T = 0: nothing to do
