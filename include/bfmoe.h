@@ -245,14 +245,18 @@ size_t bfmoe_moe_workspace_size(int d, int n_experts, int T, int k, int x_dtype)
 /*
  * Router and expert forward from and to HOST memory, the host <-> device
  * copies overlapped with the work.  The T tokens are cut into chunks of
- * `chunk` tokens, the last one taking the rest (chunk <= 0: six about equal
- * chunks of at least 2048 tokens; at most 64 chunks); chunk i's copy in,
- * chunk i-1's router + forward and chunk i-2's copy out run at the same time
- * on a library-owned copy-in stream, `stream` and a library-owned copy-out
- * stream, ordered with events.  Each token's output is that of
- * bfmoe_moe_forward on its chunk (tokens are independent; the pages route
- * every token on its own, summary 2.3).  The weight-only tables are built
- * once per call.  Pages have no counterpart for the host interface.
+ * `chunk` tokens, the last one taking the rest (chunk <= 0: T / 4096 about
+ * equal chunks, at least two and at most six, of at least 2048 tokens; at
+ * most 64 chunks).  Copies in run on a library-owned copy-in stream, copies
+ * out on a library-owned copy-out stream; the router + forward of even
+ * chunks run on `stream`, of odd chunks on a library-owned second compute
+ * stream (each of the two with its own routing buffers and scratch in ws),
+ * so that a chunk's copy in, the work of the two chunks before it and an
+ * earlier chunk's copy out overlap; events order them.  Each token's output
+ * is that of bfmoe_moe_forward on its chunk (tokens are independent; the
+ * pages route every token on its own, summary 2.3).  The weight-only tables
+ * are built once per call.  Pages have no counterpart for the host
+ * interface.
  *   x_host    host [T][d] (read), best page-locked: pageable memory makes the
  *             copies synchronous
  *   y_host    host [T][d] (written), same dtype; complete once the work
@@ -260,13 +264,14 @@ size_t bfmoe_moe_workspace_size(int d, int n_experts, int T, int k, int x_dtype)
  *             stream before reading it)
  *   chunk     tokens per chunk, or <= 0 for the default
  *   ws        device scratch of bfmoe_moe_host_workspace_size(...) bytes (the
- *             device copies of x and y, the split gate weights, one chunk's
- *             routing and one chunk's bfmoe_moe_forward scratch), 256-byte
- *             aligned
- * The copy streams and their events are created once per device on first use
- * (make that first call before any stream capture); after that the whole call
- * is stream-ordered and can be captured in a CUDA graph, copies included.
- * Calls that overlap on one device share the copy streams and serialise there.
+ *             device copies of x and y, the split gate weights, and per
+ *             compute stream one chunk's routing and one chunk's
+ *             bfmoe_moe_forward scratch), 256-byte aligned
+ * The copy and compute streams and their events are created once per device
+ * on first use (make that first call before any stream capture); after that
+ * the whole call is stream-ordered and can be captured in a CUDA graph,
+ * copies included.  Calls that overlap on one device share these streams and
+ * serialise there.
  * Returns BFMOE_EINVAL for null pointers or bad sizes, BFMOE_EWORKSPACE for a
  * short workspace.
  */

@@ -708,9 +708,12 @@ int side_stream(SideStream** out) {
 // Copy streams and events of bfmoe_moe_forward_host, one set per device,
 // created on first use.
 constexpr int kHostMaxChunks = 64;
+// `lane1` is the second compute stream: odd chunks run there, even chunks on
+// the caller's stream, so that one chunk's latency-bound kernels overlap the
+// next chunk's.
 struct HostPipe {
-  cudaStream_t in = nullptr, out = nullptr;
-  cudaEvent_t fork = nullptr, done = nullptr;
+  cudaStream_t in = nullptr, out = nullptr, lane1 = nullptr;
+  cudaEvent_t fork = nullptr, done = nullptr, lane1_go = nullptr, lane1_done = nullptr;
   cudaEvent_t ev_in[kHostMaxChunks] = {}, ev_out[kHostMaxChunks] = {};
 };
 std::mutex g_pipe_mu;
@@ -727,8 +730,11 @@ int host_pipe(HostPipe** out) {
     const unsigned ef = cudaEventDisableTiming;
     if ((e = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking)) != cudaSuccess ||
         (e = cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&hp.lane1, cudaStreamNonBlocking)) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&hp.fork, ef)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&hp.done, ef)) != cudaSuccess)
+        (e = cudaEventCreateWithFlags(&hp.done, ef)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&hp.lane1_go, ef)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&hp.lane1_done, ef)) != cudaSuccess)
       return cuda_fail(e, "moe_forward_host: copy streams");
     for (int i = 0; i < kHostMaxChunks; ++i)
       if ((e = cudaEventCreateWithFlags(&hp.ev_in[i], ef)) != cudaSuccess ||
@@ -739,21 +745,29 @@ int host_pipe(HostPipe** out) {
   return BFMOE_OK;
 }
 
-// Workspace of bfmoe_moe_forward_host: device x and y, one chunk's routing,
-// one chunk's bfmoe_moe_forward scratch; and the chunk schedule.
+// Workspace of bfmoe_moe_forward_host: device x and y, and per compute lane
+// (two when there are two chunks or more) one chunk's routing and one
+// chunk's bfmoe_moe_forward scratch; and the chunk schedule.
 struct HostPlan {
-  int chunk, nchunks;
+  int chunk, nchunks, lanes;
   int start[kHostMaxChunks + 1];  // chunk c = tokens start[c] .. start[c+1]-1
-  size_t x_dev, y_dev, idx, gates, counts, offsets, rows, parts, moe, total;
+  size_t x_dev, y_dev, parts, total;
+  size_t idx[2], gates[2], counts[2], offsets[2], rows[2], moe[2];
 };
 
 // Chunks of `chunk` tokens (the last one takes the rest).  The default is
-// six about equal chunks of at least 2048 tokens: measured on the headline
-// workload, equal chunks keep the copy-in stream, the work and the copy-out
-// stream all busy, better than a long first chunk with a tapered tail.
+// T / 4096 about equal chunks, at least two and at most six, of at least
+// 2048 tokens.  Measured end to end on B200: every chunk's work has a fixed
+// cost of about 55 us (the kernels' latency chains, nearly independent of
+// the chunk's size), so the best count balances that against the copies that
+// cannot overlap at the start and the end; four chunks at T = 16384, d = 512
+// (0.53 ms against 0.60 with six), six at T = 65536, d = 1024.
 HostPlan make_host_plan(int d, int N, int T, int k, int xdt, int chunk) {
   HostPlan h{};
-  if (chunk <= 0) chunk = std::max(2048, (T + 5) / 6);
+  if (chunk <= 0) {
+    const int want = std::min(6, std::max(2, T / 4096));
+    chunk = std::max(2048, (T + want - 1) / want);
+  }
   chunk = (chunk + 127) / 128 * 128;
   if (T > 0 && chunk > T) chunk = T;
   if (T > 0 && (T + chunk - 1) / chunk > kHostMaxChunks) chunk = (T + kHostMaxChunks - 1) / kHostMaxChunks;
@@ -778,14 +792,17 @@ HostPlan make_host_plan(int d, int N, int T, int k, int xdt, int chunk) {
   };
   h.x_dev = take(static_cast<size_t>(T) * d * es);
   h.y_dev = take(static_cast<size_t>(T) * d * es);
-  h.idx = take(rc * 4);
-  h.gates = take(rc * 4);
-  h.counts = take(static_cast<size_t>(N) * 4);
-  h.offsets = take(static_cast<size_t>(N + 1) * 4);
-  h.rows = take(rc * 4);
   h.parts = take(static_cast<size_t>(3) * N * d * 2);  // W_g split once per call (tensor-core router)
   const Plan p = make_plan(d, N, h.chunk, k, xdt);
-  h.moe = take(p.fwd_end + p.rt_end);
+  h.lanes = h.nchunks >= 2 ? 2 : 1;
+  for (int l = 0; l < h.lanes; ++l) {
+    h.idx[l] = take(rc * 4);
+    h.gates[l] = take(rc * 4);
+    h.counts[l] = take(static_cast<size_t>(N) * 4);
+    h.offsets[l] = take(static_cast<size_t>(N + 1) * 4);
+    h.rows[l] = take(rc * 4);
+    h.moe[l] = take(p.fwd_end + p.rt_end);
+  }
   h.total = off;
   return h;
 }
@@ -1232,15 +1249,12 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
   const size_t row_bytes = static_cast<size_t>(d) * (bf16 ? 2 : 4);
   uint8_t* x_dev = W + hp.x_dev;
   uint8_t* y_dev = W + hp.y_dev;
-  int32_t* idx = reinterpret_cast<int32_t*>(W + hp.idx);
-  float* gates = reinterpret_cast<float*>(W + hp.gates);
-  int32_t* counts = reinterpret_cast<int32_t*>(W + hp.counts);
-  int32_t* offsets = reinterpret_cast<int32_t*>(W + hp.offsets);
-  int32_t* rows = reinterpret_cast<int32_t*>(W + hp.rows);
-  uint8_t* Wm = W + hp.moe;
   const Plan pc = make_plan(d, N, hp.chunk, k, x_dtype);
   const uint8_t* xh = static_cast<const uint8_t*>(x_host);
   uint8_t* yh = static_cast<uint8_t*>(y_host);
+  // chunk c runs on lane c % lanes: lane 0 is `stream`, lane 1 the pipe's
+  // second compute stream, each with its own routing buffers and scratch
+  cudaStream_t lane_s[2] = {s, pipe->lane1};
 
   // the copy streams start after all earlier work on `stream` (so a previous
   // call's buffers are free); the weight tables build on the side stream
@@ -1252,8 +1266,9 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
   if (e != cudaSuccess) return cuda_fail(e, "moe_forward_host: fork");
   const uint8_t* tabs = static_cast<const uint8_t*>(layer->tables);
   if (!tabs) {
-    rc = build_weight_tables(layer, Wm + pc.tabs, ss->stream);
-    tabs = Wm + pc.tabs;
+    // (in lane 0's scratch; both lanes read them)
+    rc = build_weight_tables(layer, W + hp.moe[0] + pc.tabs, ss->stream);
+    tabs = W + hp.moe[0] + pc.tabs;
   }
   if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return cuda_fail(e, "moe_forward_host: join record");
   // W_g is split once for all chunks, while the first chunk is copied in
@@ -1267,12 +1282,26 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
       parts = own;
     }
   }
+  // lane 1 starts after the split (and so after the fork)
+  if (rc == BFMOE_OK && hp.lanes == 2 &&
+      ((e = cudaEventRecord(pipe->lane1_go, s)) != cudaSuccess ||
+       (e = cudaStreamWaitEvent(pipe->lane1, pipe->lane1_go, 0)) != cudaSuccess))
+    rc = cuda_fail(e, "moe_forward_host: lane fork");
+  const bool lane1_used = rc == BFMOE_OK && hp.lanes == 2;
   for (int c = 0; c < hp.nchunks && rc == BFMOE_OK; ++c) {
+    const int l = c % hp.lanes;
+    cudaStream_t ls = lane_s[l];
+    int32_t* idx = reinterpret_cast<int32_t*>(W + hp.idx[l]);
+    float* gates = reinterpret_cast<float*>(W + hp.gates[l]);
+    int32_t* counts = reinterpret_cast<int32_t*>(W + hp.counts[l]);
+    int32_t* offsets = reinterpret_cast<int32_t*>(W + hp.offsets[l]);
+    int32_t* rows = reinterpret_cast<int32_t*>(W + hp.rows[l]);
+    uint8_t* Wm = W + hp.moe[l];
     const int t0 = hp.start[c], Tc = hp.start[c + 1] - t0;
     const size_t o = static_cast<size_t>(t0) * row_bytes, n = static_cast<size_t>(Tc) * row_bytes;
     if ((e = cudaMemcpyAsync(x_dev + o, xh + o, n, cudaMemcpyHostToDevice, pipe->in)) != cudaSuccess ||
         (e = cudaEventRecord(pipe->ev_in[c], pipe->in)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(s, pipe->ev_in[c], 0)) != cudaSuccess) {
+        (e = cudaStreamWaitEvent(ls, pipe->ev_in[c], 0)) != cudaSuccess) {
       rc = cuda_fail(e, "moe_forward_host: copy in");
       break;
     }
@@ -1280,21 +1309,25 @@ int bfmoe_moe_forward_host(const bfmoe_layer* layer, const void* x_host, int x_d
     const Plan pcur = make_plan(d, N, Tc, k, x_dtype);
     const bool fused = fused_path(x_dtype, d);
     rc = router_topk_impl(x_dev + o, x_dtype, Tc, d, w_gate, bias, N, k, idx, gates, counts, offsets, rows,
-                          Wm + pc.fwd_end, pc.rt_end, s, parts,
+                          Wm + pc.fwd_end, pc.rt_end, ls, parts,
                           fused ? reinterpret_cast<int32_t*>(Wm + pcur.pad) : nullptr);
-    if (c == 0 && (e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) rc = cuda_fail(e, "moe_forward_host: join");
+    // each lane's first forward waits for the weight tables
+    if (c < hp.lanes && (e = cudaStreamWaitEvent(ls, ss->join, 0)) != cudaSuccess)
+      rc = cuda_fail(e, "moe_forward_host: join");
     if (rc) break;
-    rc = forward_body(layer, x_dev + o, bf16, Tc, k, idx, gates, offsets, rows, y_dev + o, pcur, Wm, tabs, s, fused);
+    rc = forward_body(layer, x_dev + o, bf16, Tc, k, idx, gates, offsets, rows, y_dev + o, pcur, Wm, tabs, ls, fused);
     if (rc) break;
-    if ((e = cudaEventRecord(pipe->ev_out[c], s)) != cudaSuccess ||
+    if ((e = cudaEventRecord(pipe->ev_out[c], ls)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(pipe->out, pipe->ev_out[c], 0)) != cudaSuccess ||
         (e = cudaMemcpyAsync(yh + o, y_dev + o, n, cudaMemcpyDeviceToHost, pipe->out)) != cudaSuccess)
       rc = cuda_fail(e, "moe_forward_host: copy out");
   }
-  // join: later work on `stream` runs after every copy out (and the side
-  // stream's tables, joined above or here when no chunk ran)
+  // join: later work on `stream` runs after every copy out, lane 1's work
+  // and the side stream's tables (joined above or here when no chunk ran)
   if ((e = cudaEventRecord(pipe->done, pipe->out)) == cudaSuccess) e = cudaStreamWaitEvent(s, pipe->done, 0);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
+  if (e == cudaSuccess && lane1_used && (e = cudaEventRecord(pipe->lane1_done, pipe->lane1)) == cudaSuccess)
+    e = cudaStreamWaitEvent(s, pipe->lane1_done, 0);
   if (e == cudaSuccess && (e = cudaEventRecord(pipe->fork, pipe->in)) == cudaSuccess)
     e = cudaStreamWaitEvent(s, pipe->fork, 0);
   if (e != cudaSuccess && rc == BFMOE_OK) rc = cuda_fail(e, "moe_forward_host: final join");
