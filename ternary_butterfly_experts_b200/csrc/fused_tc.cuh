@@ -21,12 +21,13 @@
 //                 into one fp32 accumulator of d TMEM columns: the tile's full
 //                 output rows;
 //   warps 10..17  (epilogue, two per TMEM lane quadrant, one thread per row)
-//                 apply alpha and B(phi_e) with tensor memory as the row's
-//                 fp32 backing store: stages 0..4 act inside each 32-column
-//                 chunk (tcgen05.ld, rotate, tcgen05.st); stages 5..L-1 act
-//                 on column slices c, c+32, c+64, ... loaded two slices at a
-//                 time; finally the gated row is rounded to bf16 and stored
-//                 with 32-byte stores.
+//                 apply B(phi_e) with tensor memory as the row's fp32
+//                 backing store: stages 0..4 act inside each 32-column chunk
+//                 (tcgen05.ld, rotate, tcgen05.st); stages 5..L-1 act on
+//                 column slices c, c+32, c+64, ... loaded two slices at a
+//                 time; finally the row times gate * alpha (the butterfly is
+//                 linear: g B(phi)(alpha z) = (g alpha) B(phi) z) is rounded
+//                 to bf16 and stored with 32-byte stores.
 // A (128 x d bf16) and the accumulator (128 x d fp32) fill most of shared and
 // tensor memory at d = 512, so a tile's MMAs wait for the previous tile's
 // epilogue, and the producers refill A once the previous tile's MMAs have
@@ -505,7 +506,7 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
       if (!produce_tile<D>(pc, t, i, i >= 1, buf, lane))
         break;
   } else {
-    // ---- epilogue: alpha, B(phi), gate; one thread per row ---------------
+    // ---- epilogue: B(phi), then gate * alpha; one thread per row ----------
     const int qd = warp & 3;                                  // TMEM lane quadrant
     const int ew = warp - 2 - kFusedProdWarps;                // epilogue warp 0..7
     const int wq = ew >> 2;                                   // which half of the work
@@ -521,7 +522,7 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
       i = -1;
     for (long long t = blockIdx.x; t < n_tiles && i >= 0; t += gridDim.x, ++i) {
       const PadRow pr = pad_row(t * kGemmBM + m, pmap, qex);
-      const RowMeta mt{pr.row, pr.e, pr.row >= 0 ? gates[pr.row] : 0.f};
+      const RowMeta mt{pr.row, pr.e, pr.row >= 0 ? gates[pr.row] * alpha : 0.f};
       const float4* tp = pq_phi + static_cast<size_t>(mt.ex >= 0 ? mt.ex : 0) * C::L * (D / 4);
       // the quadrant's rows share one expert (padded buckets): its quads are
       // staged into shared memory ahead of use, bypassing L1; else (past the
@@ -574,7 +575,7 @@ __global__ __launch_bounds__(kFusedThreads, 1) void fused_expert_kernel(
         tmem_wait_ld();
         float v[32];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = alpha * __uint_as_float(r[q]);
+        for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(r[q]);
         if (uni) epi_chunk_stages<D, true>(v, ebuf + b * C::EPI_QUADS, 8);
         else epi_chunk_stages<D, false>(v, tp + 8 * j, D / 4);
 #pragma unroll
