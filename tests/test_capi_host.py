@@ -83,10 +83,13 @@ def test_host_workspace_size(L):
     bf = capi.BFMOE_BF16
     full = L.bfmoe_moe_host_workspace_size(512, 256, 16384, 2, bf, 0)
     one = L.bfmoe_moe_workspace_size(512, 256, 2816, 2, bf)
-    # device x and y for all tokens plus one default chunk (T/6, rounded up
-    # to 128 tokens) of scratch
-    assert full >= 2 * 16384 * 512 * 2 + one and full % 256 == 0
-    assert L.bfmoe_moe_host_workspace_size(512, 256, 16384, 2, bf, 16384) > full  # one big chunk needs more
+    # device x and y for all tokens plus, per compute stream, one default
+    # chunk's scratch (four chunks of 4096 tokens here, two streams)
+    assert full >= 2 * 16384 * 512 * 2 + 2 * L.bfmoe_moe_workspace_size(512, 256, 4096, 2, bf) and full % 256 == 0
+    assert full >= 2 * 16384 * 512 * 2 + one
+    # one chunk of all tokens: one compute stream with the whole call's scratch
+    big = L.bfmoe_moe_host_workspace_size(512, 256, 16384, 2, bf, 16384)
+    assert big >= 2 * 16384 * 512 * 2 + L.bfmoe_moe_workspace_size(512, 256, 16384, 2, bf)
     assert L.bfmoe_moe_host_workspace_size(500, 256, 16384, 2, bf, 0) == 0
     assert L.bfmoe_moe_host_workspace_size(512, 4, 100, 5, bf, 0) == 0
 
